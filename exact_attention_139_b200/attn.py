@@ -1,0 +1,197 @@
+"""Thin ctypes binding of libattn_b200.so (C ABI in include/attn.h).
+
+Argument marshalling only: shapes are read from the torch tensors, device pointers and the
+current CUDA stream are passed through, and every step of the computation runs in the CUDA
+library. Importing this module raises if the library has not been built; there is no fallback.
+
+Functions keep the C names:
+    attn_fwd(q, k, v, causal=..., scale=None, out=None, lse=None)          -> (o, lse)
+    attn_decode(q, k, v, causal=..., dv=None, num_splits=0, impl=0, ...)   -> (o, lse)
+    attn_combine(o_part, lse_part, out=None, lse=None)                     -> (o, lse)
+    attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)         -> int
+    attn_status_string(code), attn_check_device(), attn_selftest_wait_timeout(limit_us)
+plus attn_fwd_host(...): host tensors in, host tensors out (pinned copies around attn_fwd).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_attention_139_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_lib.attn_fwd.restype = _i
+_lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _vp]
+_lib.attn_decode_workspace_size.restype = _sz
+_lib.attn_decode_workspace_size.argtypes = [_i] * 7
+_lib.attn_decode.restype = _i
+_lib.attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _sz, _vp]
+_lib.attn_decode_ex.restype = _i
+_lib.attn_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _sz, _i, _vp]
+_lib.attn_combine.restype = _i
+_lib.attn_combine.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp]
+_lib.attn_decode_default_splits.restype = _i
+_lib.attn_decode_default_splits.argtypes = [_i] * 7
+_lib.attn_check_device.restype = _i
+_lib.attn_check_device.argtypes = [_vp]
+_lib.attn_selftest_wait_timeout.restype = _i
+_lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
+_lib.attn_status_string.restype = ctypes.c_char_p
+_lib.attn_status_string.argtypes = [_i]
+_lib.attn_abi_version.restype = _i
+_lib.attn_abi_version.argtypes = []
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED = 0, 1, 2, 3
+ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = 4, 5, 6
+ATTN_DECODE_AUTO, ATTN_DECODE_CUDA_CORE, ATTN_DECODE_TCGEN05_T = 0, 1, 2
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {attn_status_string(code)} (status {code})")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def attn_status_string(code: int) -> str:
+    return _lib.attn_status_string(int(code)).decode()
+
+
+def attn_abi_version() -> int:
+    return _lib.attn_abi_version()
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(code: int, where: str):
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
+             out: torch.Tensor | None = None, lse: torch.Tensor | None = None, want_lse: bool = True):
+    """O [B,Hq,Lq,dv] bf16 and LSE [B,Hq,Lq] fp32 for q [B,Hq,Lq,d], k/v [B,Hkv,Lk,d/dv]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dv = v.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    code = _lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
+                         scale, int(bool(causal)), _stream_handle(q.device))
+    _check(code, "attn_fwd")
+    return out, lse
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits=0) -> int:
+    return int(_lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits))
+
+
+def attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv) -> int:
+    return int(_lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv))
+
+
+def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
+                dv: int | None = None, num_splits: int = 0, impl: int = ATTN_DECODE_AUTO,
+                workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None):
+    """Split-KV decode. ``v is k`` selects the latent layout (V = first ``dv`` columns of K)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    ldv = v.shape[-1]
+    dv = ldv if dv is None else int(dv)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    need = attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    code = _lib.attn_decode_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, int(bool(causal)), int(num_splits),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(impl),
+                               _stream_handle(q.device))
+    _check(code, "attn_decode")
+    return out, lse
+
+
+def attn_combine(o_part: torch.Tensor, lse_part: torch.Tensor, *, B: int, Hq: int, Lq: int,
+                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """o_part fp32 [S, B*Hq*Lq, dv], lse_part fp32 [S, B*Hq*Lq] -> O bf16 [B,Hq,Lq,dv], LSE."""
+    _need(o_part, "o_part", torch.float32)
+    _need(lse_part, "lse_part", torch.float32)
+    S, rows, dv = o_part.shape
+    if out is None:
+        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=o_part.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=o_part.device)
+    code = _lib.attn_combine(o_part.data_ptr(), lse_part.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, Hq, Lq, dv, S, _stream_handle(o_part.device))
+    _check(code, "attn_combine")
+    return out, lse
+
+
+def attn_check_device(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device error status."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return int(_lib.attn_check_device(_stream_handle(dev)))
+
+
+def attn_selftest_wait_timeout(limit_us: int, device=None):
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check(_lib.attn_selftest_wait_timeout(int(limit_us), _stream_handle(dev)), "attn_selftest_wait_timeout")
+
+
+def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
+                  device="cuda:0", bufs: dict | None = None):
+    """Host (CPU, ideally pinned) tensors in, host tensors out: copy in, attn_fwd, copy out.
+
+    ``bufs`` may hold reusable device / pinned buffers (keys q, k, v, o, lse, o_host, lse_host)."""
+    dev = torch.device(device)
+    bufs = {} if bufs is None else bufs
+    B, Hq, Lq, d = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if name not in bufs:
+            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
+        bufs[name].copy_(t, non_blocking=True)
+    if "o" not in bufs:
+        bufs["o"] = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=dev)
+        bufs["lse"] = torch.empty((B, Hq, Lq), dtype=torch.float32, device=dev)
+        bufs["o_host"] = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, pin_memory=True)
+        bufs["lse_host"] = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
+    attn_fwd(bufs["q"], bufs["k"], bufs["v"], causal=causal, scale=scale, out=bufs["o"], lse=bufs["lse"])
+    bufs["o_host"].copy_(bufs["o"], non_blocking=True)
+    bufs["lse_host"].copy_(bufs["lse"], non_blocking=True)
+    torch.cuda.current_stream(dev).synchronize()
+    return bufs["o_host"], bufs["lse_host"]

@@ -1,0 +1,391 @@
+// attn_api.cu -- the C ABI of libattn_b200.so (declared in include/attn.h).
+//
+// Host side only: argument checks, TMA tensor-map encoding (driver entry point looked up once),
+// split selection and kernel launches. The kernels live in the .cuh files included below so the
+// whole library is one translation unit (one device-side error word, no device linking).
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/attn.h"
+#include "combine.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using attn::DecodeParams;
+using attn::PrefillParams;
+
+constexpr int kAbiVersion = 10000;  // 1.0.0
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map over a row-major [n2, n1, n0] array (n0 contiguous), 128-byte swizzle,
+// zero fill out of bounds. box = {b0, b1, 1}. rank 2 when n2 == 0.
+bool encode_bf16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {n0, n1, n2};
+  cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = n2 == 0 ? 2 : 3;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// Set the dynamic shared-memory limit of a kernel (cheap; done on every launch so that every
+// device the caller uses is covered).
+template <typename K>
+bool allow_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+attn_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
+                         int Hkv, int Lq, int Lk, int d, int dv, float scale, int causal) {
+  if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || d < 1 || dv < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq > 0x7fffffffLL || (long long)B * Hq * Lq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return ATTN_ERR_MISALIGNED;
+  if (lse && !aligned(lse, 4)) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// decode: split selection and workspace layout
+// ---------------------------------------------------------------------------------------------
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t workspace_bytes(long long rows, int dv, int splits) {
+  return align256((size_t)splits * rows * dv * 4) + align256((size_t)splits * rows * 4);
+}
+
+bool tc_supported(const void* k, const void* v, int Hq, int Hkv, int Lq, int d, int dv, int ldv) {
+  const int R = (Hq / Hkv) * Lq;
+  return v == k && ldv == d && d % 64 == 0 && d <= 576 && dv % 128 == 0 && dv <= 512 && dv <= d && R <= 32;
+}
+
+bool cc_supported(int Hq, int Hkv, int Lq, int d, int dv, int ldv) {
+  const int R = (Hq / Hkv) * Lq;
+  return R <= 64 && d <= 576 && dv <= 512 && d % 8 == 0 && dv % 8 == 0 && ldv % 8 == 0 && ldv >= dv;
+}
+
+// Keys per split: a multiple of 64.
+int split_chunk(int Lk, int splits) {
+  int c = (Lk + splits - 1) / splits;
+  return (c + 63) / 64 * 64;
+}
+
+// Choose the split count: every CTA is resident one per SM (tensor-core kernel) or a few per SM
+// (CUDA-core kernel); minimise idle SMs in the last wave plus the partial-result traffic relative
+// to the KV bytes, with at least 256 keys per split.
+// Depends only on the sizes attn_decode_workspace_size also sees (the KV bytes are estimated
+// from dv), so both always agree on the count.
+int choose_splits(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int sms, int ctas_per_sm) {
+  const long long units = (long long)B * Hkv;
+  const long long rows = (long long)B * Hq * Lq;
+  const double kv_bytes = (double)units * Lk * (double)dv * 2.0;
+  const int max_s = std::max(1, std::min(256, Lk / 256));
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= max_s; ++s) {
+    const int chunk = split_chunk(Lk, s);
+    const int used = (Lk + chunk - 1) / chunk;  // splits that hold keys
+    if (used < s) continue;
+    const double slots = (double)sms * ctas_per_sm;
+    const double waves = (double)(units * s) / slots;
+    const double waste = std::ceil(waves) / waves - 1.0;
+    const double partial = 2.0 * (double)s * rows * (dv + 1) * 4.0 / kv_bytes;
+    const double cost = waste + partial + (waves < 1.0 ? (1.0 - waves) : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+template <int RMAX, int CPT>
+attn_status launch_cc(const DecodeParams& p, int splits, cudaStream_t st) {
+  const size_t smem = attn::decode_cc_smem_bytes(p.R, p.d, p.dv, !p.v_is_k);
+  auto kern = attn::decode_cc_kernel<RMAX, CPT>;
+  if (smem > 48 * 1024 && !allow_smem(kern, (int)smem)) return ATTN_ERR_CUDA;
+  dim3 grid(splits, p.B * p.Hkv);
+  kern<<<grid, attn::kCcThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+template <int DCH, int NB, int NP>
+attn_status launch_tc(const DecodeParams& p, int splits, cudaStream_t st) {
+  using C = attn::DecodeTcCfg<DCH, NB, NP>;
+  CUtensorMap tq, tkv;
+  if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, NP)) return ATTN_ERR_CUDA;
+  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, C::BKV)) return ATTN_ERR_CUDA;
+  auto kern = attn::decode_tc_kernel<DCH, NB, NP>;
+  if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  dim3 grid(splits, p.B * p.Hkv);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, p);
+  return launch_status();
+}
+
+template <int DCH, int NB>
+attn_status launch_tc_np(const DecodeParams& p, int splits, cudaStream_t st) {
+  if (p.R <= 16) return launch_tc<DCH, NB, 16>(p, splits, st);
+  return launch_tc<DCH, NB, 32>(p, splits, st);
+}
+
+template <int DCH>
+attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
+  switch (p.dv / 128) {
+    // V^T block nb reads 64-column chunks 2nb and 2nb+1 of the latent tile, so 2*NB <= DCH
+    case 1: if constexpr (2 <= DCH) return launch_tc_np<DCH, 1>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 2: if constexpr (4 <= DCH) return launch_tc_np<DCH, 2>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 3: if constexpr (6 <= DCH) return launch_tc_np<DCH, 3>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 4: if constexpr (8 <= DCH) return launch_tc_np<DCH, 4>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+attn_status launch_tc_any(const DecodeParams& p, int splits, cudaStream_t st) {
+  switch (p.d / 64) {
+    case 2: return launch_tc_nb<2>(p, splits, st);
+    case 3: return launch_tc_nb<3>(p, splits, st);
+    case 4: return launch_tc_nb<4>(p, splits, st);
+    case 5: return launch_tc_nb<5>(p, splits, st);
+    case 6: return launch_tc_nb<6>(p, splits, st);
+    case 7: return launch_tc_nb<7>(p, splits, st);
+    case 8: return launch_tc_nb<8>(p, splits, st);
+    case 9: return launch_tc_nb<9>(p, splits, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+attn_status launch_combine(const float* o_part, const float* lse_part, void* o, float* lse, long long rows, int dv,
+                           int splits, cudaStream_t st) {
+  if (rows <= 0) return ATTN_OK;
+  attn::combine_kernel<<<(unsigned)rows, attn::kCombineThreads, 0, st>>>(
+      o_part, lse_part, reinterpret_cast<__nv_bfloat16*>(o), lse, rows, dv, splits);
+  return launch_status();
+}
+
+// One CTA waits on a barrier that never completes; the bounded wait gives up after limit_ns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = attn::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    attn::mbar_init(b, 1);
+    attn::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!attn::mbar_try_wait(b, 0)) (void)attn::mbar_wait_slow(b, 0, 0xEE, limit_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case ATTN_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "a bounded wait on the GPU ran out";
+  }
+  return "unknown status";
+}
+
+int attn_abi_version(void) { return kAbiVersion; }
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                     int Lk, int d, int dv, float scale, int causal, void* stream) {
+  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+  PrefillParams p{};
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (Lq + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long grid = (long long)p.n_qtiles * B * Hq;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128) {
+    using C = attn::PrefillCfg<128>;
+    if (!encode_bf16(&tq, q, 128, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
+        !encode_bf16(&tk, k, 128, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
+        !encode_bf16(&tv, v, 128, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
+      return ATTN_ERR_CUDA;
+    if (!allow_smem(attn::prefill_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill_kernel<128><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+  } else {
+    using C = attn::PrefillCfg<64>;
+    if (!encode_bf16(&tq, q, 64, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
+        !encode_bf16(&tk, k, 64, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
+        !encode_bf16(&tv, v, 64, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
+      return ATTN_ERR_CUDA;
+    if (!allow_smem(attn::prefill_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill_kernel<64><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+  }
+  return launch_status();
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || dv < 1 || num_splits < 0 || num_splits > 256) return 0;
+  if (Hq % Hkv != 0) return 0;
+  int s = num_splits;
+  if (s == 0) s = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  return workspace_bytes((long long)B * Hq * Lq, dv, s);
+}
+
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
+  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+}
+
+attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                           void* workspace, size_t ws_bytes, int impl, void* stream) {
+  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (ldv < dv) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
+  if (impl < ATTN_DECODE_AUTO || impl > ATTN_DECODE_TCGEN05_T) return ATTN_ERR_INVALID_ARG;
+  if (d % 8 != 0 || dv % 8 != 0 || ldv % 8 != 0) return ATTN_ERR_MISALIGNED;
+  const bool tc_ok = tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
+  const bool cc_ok = cc_supported(Hq, Hkv, Lq, d, dv, ldv);
+  if (impl == ATTN_DECODE_AUTO) impl = tc_ok ? ATTN_DECODE_TCGEN05_T : ATTN_DECODE_CUDA_CORE;
+  if (impl == ATTN_DECODE_TCGEN05_T && !tc_ok) return ATTN_ERR_UNSUPPORTED;
+  if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
+  int splits = num_splits;
+  if (splits == 0) splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  const long long rows = (long long)B * Hq * Lq;
+  const size_t need = workspace_bytes(rows, dv, splits);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
+
+  DecodeParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.o_part = reinterpret_cast<float*>(workspace);
+  p.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + align256((size_t)splits * rows * dv * 4));
+  p.rows_total = rows;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.d = d;
+  p.dv = dv;
+  p.ldv = ldv;
+  p.G = Hq / Hkv;
+  p.R = p.G * Lq;
+  p.causal = causal ? 1 : 0;
+  p.chunk = split_chunk(Lk, splits);
+  p.v_is_k = (v == k && ldv == d) ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  if (impl == ATTN_DECODE_TCGEN05_T) {
+    st = launch_tc_any(p, splits, cs);
+  } else {
+    const int cpt = (dv + attn::kCcThreads - 1) / attn::kCcThreads;
+    if (p.R <= 16) st = cpt == 1 ? launch_cc<16, 1>(p, splits, cs) : launch_cc<16, 2>(p, splits, cs);
+    else if (p.R <= 32) st = cpt == 1 ? launch_cc<32, 1>(p, splits, cs) : launch_cc<32, 2>(p, splits, cs);
+    else st = cpt == 1 ? launch_cc<64, 1>(p, splits, cs) : launch_cc<64, 2>(p, splits, cs);
+  }
+  if (st != ATTN_OK) return st;
+  return launch_combine(p.o_part, p.lse_part, o, lse, rows, dv, splits, cs);
+}
+
+attn_status attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  return attn_decode_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits, workspace,
+                        ws_bytes, ATTN_DECODE_AUTO, stream);
+}
+
+attn_status attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq, int Lq,
+                         int dv, int num_splits, void* stream) {
+  if (!o_part || !lse_part || !o) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Lq < 1 || dv < 1 || num_splits < 1 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+  if (dv % 4 != 0) return ATTN_ERR_MISALIGNED;
+  if (!aligned(o_part, 16) || !aligned(lse_part, 4) || !aligned(o, 8) || (lse && !aligned(lse, 4)))
+    return ATTN_ERR_MISALIGNED;
+  const long long rows = (long long)B * Hq * Lq;
+  if (rows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  return launch_combine(o_part, lse_part, o, lse, rows, dv, num_splits, reinterpret_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull);
+  return launch_status();
+}
+
+attn_status attn_check_device(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, attn::g_attn_dev_error, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(attn::g_attn_dev_error, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

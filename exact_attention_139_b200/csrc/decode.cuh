@@ -1,0 +1,558 @@
+// decode.cuh -- split-KV decode attention (few query tokens, long KV cache) on sm_100a.
+//
+// Each CTA takes one (batch, kv head, key chunk) and computes, for the R = (Hq/Hkv)*Lq query
+// rows that share the kv head, a partial O over its chunk (fp32, divided by its own softmax
+// sum) and the chunk's LSE (natural log; -inf when no key of the chunk is visible). The
+// log-sum-exp combine (combine.cuh) merges the chunks.
+//
+// Two kernels:
+//   decode_cc_kernel      fp32 CUDA-core dot products; any supported shape; the baseline.
+//   decode_tc_kernel      tcgen05 with the key length on the MMA M dimension: the transposed
+//                         flow S^T = K.Q^T, P^T = softmax(S^T), O^T = V^T.P^T of the FlashMLA-ETAP
+//                         summary ("Mecanismo Central", items 1-3). With only R = 32 query rows
+//                         per kv head, putting keys (64 per tile) on M and queries on N avoids
+//                         padding the query dimension to the MMA's minimum M.
+// Latent KV (MLA): V is the first dv columns of each K row; each row is read from HBM once and
+// the same shared-memory tile feeds both products.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  float* o_part;    // [num_splits, rows_total, dv]
+  float* lse_part;  // [num_splits, rows_total]
+  long long rows_total;
+  int B, Hq, Hkv, Lq, Lk, d, dv, ldv, G, R;
+  int causal;
+  int chunk;  // keys per split (multiple of 64)
+  int v_is_k;
+  float scale_log2;
+};
+
+// ======================================================================================
+// CUDA-core kernel
+// ======================================================================================
+constexpr int kCcKeys = 32;      // keys per shared-memory chunk
+constexpr int kCcThreads = 256;
+
+__host__ __device__ inline int cc_row_stride(int n) { return n + 8; }  // pad rows by 16 bytes
+
+__host__ inline size_t decode_cc_smem_bytes(int R, int d, int dv, bool separate_v) {
+  size_t b = (size_t)R * d * 2;                                   // Q (bf16)
+  b += (size_t)kCcKeys * cc_row_stride(d) * 2;                    // K chunk
+  if (separate_v) b += (size_t)kCcKeys * cc_row_stride(dv) * 2;   // V chunk
+  b += (size_t)64 * kCcKeys * 4;                                  // scores / probabilities
+  b += 64 * 4 * 2;                                                // alpha, l
+  return b;
+}
+
+template <int RMAX, int CPT>
+__global__ void __launch_bounds__(kCcThreads)
+    decode_cc_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int split = blockIdx.x;
+  const int unit = blockIdx.y;
+  const int b = unit / p.Hkv, hkv = unit % p.Hkv;
+  const int tid = threadIdx.x;
+  const int R = p.R;
+  const int ks = cc_row_stride(p.d), vs = cc_row_stride(p.dv);
+  const bool sep_v = !p.v_is_k;
+
+  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* Ks = Qs + (size_t)R * p.d;
+  __nv_bfloat16* Vs = Ks + (size_t)kCcKeys * ks;
+  float* Ss = reinterpret_cast<float*>(Vs + (sep_v ? (size_t)kCcKeys * vs : 0));
+  float* alpha_s = Ss + 64 * kCcKeys;
+  float* l_s = alpha_s + 64;
+
+  const long long row0 = ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
+  const int j_begin = split * p.chunk;
+  const int j_end = min(p.Lk, j_begin + p.chunk);
+  const int off = p.Lk - p.Lq;
+
+  // Q rows of this kv head are contiguous: [R, d]
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + row0 * p.d);
+    uint4* dst = reinterpret_cast<uint4*>(Qs);
+    for (int i = tid; i < R * p.d / 8; i += kCcThreads) dst[i] = src[i];
+  }
+  float acc[RMAX][CPT];
+#pragma unroll
+  for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+    for (int cc = 0; cc < CPT; ++cc) acc[r][cc] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // meaningful in threads tid < R
+
+  const __nv_bfloat16* kbase = p.k + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.d;
+  const __nv_bfloat16* vbase = p.v + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.ldv;
+
+  for (int kc = j_begin; kc < j_end; kc += kCcKeys) {
+    __syncthreads();  // previous chunk fully consumed
+    const int nk = min(kCcKeys, j_end - kc);
+    for (int i = tid; i < kCcKeys * (p.d / 8); i += kCcThreads) {
+      const int jr = i / (p.d / 8), u = i % (p.d / 8);
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (jr < nk) val = *reinterpret_cast<const uint4*>(kbase + (long long)(kc + jr) * p.d + 8 * u);
+      *reinterpret_cast<uint4*>(Ks + jr * ks + 8 * u) = val;
+    }
+    if (sep_v) {
+      for (int i = tid; i < kCcKeys * (p.dv / 8); i += kCcThreads) {
+        const int jr = i / (p.dv / 8), u = i % (p.dv / 8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (jr < nk) val = *reinterpret_cast<const uint4*>(vbase + (long long)(kc + jr) * p.ldv + 8 * u);
+        *reinterpret_cast<uint4*>(Vs + jr * vs + 8 * u) = val;
+      }
+    }
+    __syncthreads();
+    // scores: pairs (r, jr)
+    for (int idx = tid; idx < R * kCcKeys; idx += kCcThreads) {
+      const int r = idx / kCcKeys, jr = idx % kCcKeys;
+      const int key = kc + jr;
+      const int i = r % p.Lq;
+      float sc = -INFINITY;
+      if (jr < nk && (!p.causal || key <= i + off)) {
+        const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(Qs + r * p.d);
+        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(Ks + jr * ks);
+        float a0 = 0.f, a1 = 0.f;
+        for (int c = 0; c < p.d / 2; ++c) {
+          const float2 qf = __bfloat1622float2(qr[c]);
+          const float2 kf = __bfloat1622float2(kr[c]);
+          a0 = fmaf(qf.x, kf.x, a0);
+          a1 = fmaf(qf.y, kf.y, a1);
+        }
+        sc = a0 + a1;
+      }
+      Ss[r * kCcKeys + jr] = sc;
+    }
+    __syncthreads();
+    if (tid < R) {
+      float mx = -INFINITY;
+      for (int jr = 0; jr < kCcKeys; ++jr) mx = fmaxf(mx, Ss[tid * kCcKeys + jr]);
+      const float m_tile = mx * p.scale_log2;
+      float alpha = 1.f;
+      if (m_tile != -INFINITY && (m_run == -INFINITY || m_tile > m_run + kRescaleLog2)) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
+        m_run = m_tile;
+      }
+      float sum = 0.f;
+      for (int jr = 0; jr < kCcKeys; ++jr) {
+        const float sc = Ss[tid * kCcKeys + jr];
+        const float pr = (sc == -INFINITY) ? 0.f : ex2_approx(fmaf(sc, p.scale_log2, -m_run));
+        Ss[tid * kCcKeys + jr] = pr;
+        sum += pr;
+      }
+      l_run = l_run * alpha + sum;
+      alpha_s[tid] = alpha;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+      if (r < R) {
+        const float a = alpha_s[r];
+#pragma unroll
+        for (int cc = 0; cc < CPT; ++cc) acc[r][cc] *= a;
+      }
+    }
+    const __nv_bfloat16* Vsrc = sep_v ? Vs : Ks;
+    const int vstride = sep_v ? vs : ks;
+    for (int jr = 0; jr < nk; ++jr) {
+      float vv[CPT];
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc) {
+        const int c = tid + cc * kCcThreads;
+        vv[cc] = (c < p.dv) ? __bfloat162float(Vsrc[jr * vstride + c]) : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < RMAX; ++r) {
+        if (r < R) {
+          const float pr = Ss[r * kCcKeys + jr];
+#pragma unroll
+          for (int cc = 0; cc < CPT; ++cc) acc[r][cc] = fmaf(pr, vv[cc], acc[r][cc]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < R) {
+    l_s[tid] = l_run;
+    p.lse_part[(long long)split * p.rows_total + row0 + tid] =
+        (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < RMAX; ++r) {
+    if (r < R) {
+      const float lr = l_s[r];
+      const float inv = (lr > 0.f) ? 1.f / lr : 0.f;
+      float* dst = p.o_part + ((long long)split * p.rows_total + row0 + r) * p.dv;
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc) {
+        const int c = tid + cc * kCcThreads;
+        if (c < p.dv) dst[c] = acc[r][cc] * inv;
+      }
+    }
+  }
+}
+
+// ======================================================================================
+// tcgen05 kernel, key length on the MMA M dimension
+// ======================================================================================
+template <int DCH, int NB, int NP>
+struct DecodeTcCfg {
+  static constexpr int BKV = 64;                 // keys per tile (MMA M of S^T)
+  static constexpr int KCH = BKV * 128;          // one 64-row x 128-byte chunk
+  static constexpr int STAGE = DCH * KCH;        // one K tile (all d columns)
+  static constexpr int QCH = NP * 128;           // one NP-row x 128-byte chunk of Q
+  static constexpr int PT = NP * BKV * 2;        // P^T tile bf16 (no swizzle, 8x16B cores)
+  static constexpr int TROW = NP + 1;            // reduction scratch row stride (floats)
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_Q = OFF_KV + 2 * STAGE;
+  static constexpr int OFF_P = OFF_Q + DCH * QCH;
+  static constexpr int OFF_T = OFF_P + 2 * PT;
+  static constexpr int OFF_FIN = OFF_T + BKV * TROW * 4;
+  // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain, group
+  static constexpr int OFF_BAR = (OFF_FIN + 3 * NP * 4 + 7) / 8 * 8;
+  static constexpr int N_BARS = 13;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
+  static constexpr uint32_t S_COL = 0;            // S^T buffers: columns [0, 2*NP)
+  static constexpr uint32_t O_COL = 2 * NP;       // O^T blocks: NB x NP columns
+  static constexpr uint32_t TMEM_COLS = (2 * NP + NB * NP) <= 128 ? 128 : ((2 * NP + NB * NP) <= 256 ? 256 : 512);
+  static constexpr int THREADS = 192;
+  static_assert(NP == 16 || NP == 32, "query rows padded to 16 or 32");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// TMEM load of NP columns (NP = 16 or 32) for the calling warp's 32 lanes.
+template <int NP>
+__device__ __forceinline__ void tmem_ld_np(uint32_t taddr, float (&v)[32]) {
+  if constexpr (NP == 32) {
+    tmem_ld32(taddr, v);
+  } else {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+    for (int i = 16; i < 32; ++i) v[i] = 0.f;
+  }
+}
+
+template <int NP>
+__device__ __forceinline__ void tmem_st_np(uint32_t taddr, const float (&v)[32]) {
+  if constexpr (NP == 32) {
+    tmem_st32(taddr, v);
+  } else {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32"
+        " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+        : "memory");
+  }
+}
+
+template <int DCH, int NB, int NP>
+__global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                     const DecodeParams p) {
+  using C = DecodeTcCfg<DCH, NB, NP>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int split = blockIdx.x;
+  const int unit = blockIdx.y;
+  const int b = unit / p.Hkv, hkv = unit % p.Hkv;
+  const long long row0 = ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
+  const int j_begin = split * p.chunk;
+  const int j_end = min(p.Lk, j_begin + p.chunk);
+  const int n_tiles = j_end > j_begin ? (j_end - j_begin + C::BKV - 1) / C::BKV : 0;
+  const int off = p.Lk - p.Lq;
+
+  const uint32_t bar_q = base + C::OFF_BAR;
+  const uint32_t bar_kv_full = bar_q + 8;
+  const uint32_t bar_kv_empty = bar_kv_full + 16;
+  const uint32_t bar_s_full = bar_kv_empty + 16;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_pv_done = bar_p_full + 16;
+  const uint32_t bar_drain = bar_pv_done + 16;
+  const uint32_t bar_grp = bar_drain + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+  float* T = reinterpret_cast<float*>(smem + C::OFF_T);
+  float* fin_m = reinterpret_cast<float*>(smem + C::OFF_FIN);
+  float* fin_a = fin_m + NP;
+  float* fin_l = fin_a + NP;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_kv_full + 8 * i, 1);
+      mbar_init(bar_kv_empty + 8 * i, 1);
+      mbar_init(bar_s_full + 8 * i, 1);
+      mbar_init(bar_p_full + 8 * i, 128);
+      mbar_init(bar_pv_done + 8 * i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_grp, 128);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 4) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kv);
+      mbar_arrive_expect_tx(bar_q, DCH * C::QCH);
+#pragma unroll
+      for (int c = 0; c < DCH; ++c) tma_load_2d(base + C::OFF_Q + c * C::QCH, &tm_q, bar_q, 64 * c, (int)row0);
+      const int z = b * p.Hkv + hkv;
+      int t = 0;
+      bool ok = true;
+      for (; t < n_tiles; ++t) {
+        const int s = t & 1;
+        if (t >= 2) ok = mbar_wait(bar_kv_empty + 8 * s, ((t >> 1) & 1) ^ 1, 21);
+        if (!ok) break;
+        const uint32_t full = bar_kv_full + 8 * s;
+        mbar_arrive_expect_tx(full, C::STAGE);
+#pragma unroll
+        for (int c = 0; c < DCH; ++c)
+          tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * C::BKV, z);
+      }
+      if (!ok) {
+        mbar_wait_drain(bar_q, 0);
+        for (int u = max(0, t - 2); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u & 1), (u >> 1) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(64, NP, false, false);  // S^T = K.Q^T
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, NP, true, false);  // O^T += V^T.P^T
+      bool ok = mbar_wait(bar_q, 0, 22);
+      bool issued = false;
+      auto pv = [&](int tt) {
+        ok = mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 23);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KV + (tt & 1) * C::STAGE;
+        const uint32_t pb = base + C::OFF_P + (tt & 1) * C::PT;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+          for (int kk = 0; kk < C::BKV / 16; ++kk) {
+            // A = V^T block nb: dv rows [128nb, 128nb+128) = chunks 2nb, 2nb+1 (MN-major)
+            const uint64_t ad = make_sdesc(kb + (2 * nb) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
+            // B = P^T: NP x 64 keys, K-major 8x16B core matrices (LBO 128, SBO 1024)
+            const uint64_t bd = make_sdesc(pb + kk * 256, 128, 1024, kSwizzleNone);
+            mma_ss(tmem + C::O_COL + nb * NP, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_kv_empty + 8 * (tt & 1));
+        mma_commit(bar_pv_done + 8 * (tt & 1));
+      };
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        ok = mbar_wait(bar_kv_full + 8 * (t & 1), (t >> 1) & 1, 24);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KV + (t & 1) * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < 4 * DCH; ++kk) {
+          const uint64_t ad = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bd = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          mma_ss(tmem + C::S_COL + (t & 1) * NP, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        mma_commit(bar_s_full + 8 * (t & 1));
+        if (t > 0) pv(t - 1);
+      }
+      if (ok) pv(n_tiles - 1);
+      if (!ok && issued) {
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else {
+    // --------------------------- softmax warpgroup (warps 0-3) ---------------------------
+    const int tid = threadIdx.x;        // 0..127
+    const bool has_row = lane < 16;     // M = 64 layout: keys live in lanes 0-15 of each quadrant
+    const int kr = 16 * warp + lane;    // key row of the tile for has_row lanes
+    const uint32_t tw = tmem + ((uint32_t)(warp * 32) << 16);
+    constexpr int PARTS = 128 / NP;     // threads per query column in the reductions
+    constexpr int RPP = C::BKV / PARTS; // key rows per thread in the reductions
+    const int col = tid / PARTS, part = tid % PARTS;
+    const float c2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;  // of query column `col` (replicated over parts)
+    bool ok = true;
+    uint32_t gphase = 0;
+    // barrier over the 128 softmax threads with a bounded wait (a plain bar.sync cannot give up)
+    auto group_sync = [&]() -> bool {
+      mbar_arrive(bar_grp);
+      const bool r = mbar_wait(bar_grp, gphase, 29);
+      gphase ^= 1u;
+      return __all_sync(0xffffffffu, r);
+    };
+    // per-column visibility limit (causal): query column n is token i = n % Lq
+    for (int t = 0; t < n_tiles; ++t) {
+      ok = mbar_wait(bar_s_full + 8 * (t & 1), (t >> 1) & 1, 25);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float x[32];
+      tmem_ld_np<NP>(tw + C::S_COL + (t & 1) * NP, x);
+      tmem_wait_ld();
+      const int key = j_begin + t * C::BKV + kr;
+      if (has_row) {
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+          const bool vis = key < j_end && n < p.R && (!p.causal || key <= (n % p.Lq) + off);
+          T[kr * C::TROW + n] = vis ? x[n] : -INFINITY;
+        }
+      }
+      ok = group_sync();
+      if (!ok) break;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < RPP; ++i) mx = fmaxf(mx, T[(part * RPP + i) * C::TROW + col]);
+#pragma unroll
+      for (int sh = 1; sh < PARTS; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+      const float m_tile = mx * c2;
+      float alpha = 1.f;
+      if (m_tile != -INFINITY && (m_run == -INFINITY || m_tile > m_run + kRescaleLog2)) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
+        m_run = m_tile;
+      }
+      if (part == 0) {
+        fin_m[col] = m_run;
+        fin_a[col] = alpha;
+      }
+      // P^T buffer (t & 1) is free once O^T += V^T.P^T of tile t-2 has completed
+      if (t >= 2) {
+        ok = mbar_wait(bar_pv_done + 8 * (t & 1), ((t - 2) >> 1) & 1, 26);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      ok = group_sync();
+      if (!ok) break;
+      uint8_t* pbuf = smem + C::OFF_P + (t & 1) * C::PT;
+      if (has_row) {
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+          const float sv = T[kr * C::TROW + n];
+          const float mn = fin_m[n];
+          const float pr = (sv == -INFINITY) ? 0.f : ex2_approx(fmaf(sv, c2, -mn));
+          T[kr * C::TROW + n] = pr;
+          // element (n, key kr) of the K-major no-swizzle P^T tile
+          const uint32_t o = (uint32_t)(n >> 3) * 1024u + (uint32_t)(kr >> 3) * 128u +
+                             (uint32_t)(n & 7) * 16u + (uint32_t)(kr & 7) * 2u;
+          *reinterpret_cast<__nv_bfloat16*>(pbuf + o) = __float2bfloat16_rn(pr);
+        }
+      }
+      ok = group_sync();
+      if (!ok) break;
+      float sm = 0.f;
+#pragma unroll
+      for (int i = 0; i < RPP; ++i) sm += T[(part * RPP + i) * C::TROW + col];
+#pragma unroll
+      for (int sh = 1; sh < PARTS; sh <<= 1) sm += __shfl_xor_sync(0xffffffffu, sm, sh);
+      l_run = l_run * alpha + sm;
+      bool any_rescale = false;
+#pragma unroll
+      for (int n = 0; n < NP; ++n) any_rescale |= (fin_a[n] != 1.f);
+      if (any_rescale && t > 0) {
+        ok = mbar_wait(bar_pv_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, 27);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        float a[32];
+#pragma unroll
+        for (int n = 0; n < 32; ++n) a[n] = (n < NP) ? fin_a[n] : 1.f;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          float o[32];
+          tmem_ld_np<NP>(tw + C::O_COL + nb * NP, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int n = 0; n < 32; ++n) o[n] *= a[n];
+          tmem_st_np<NP>(tw + C::O_COL + nb * NP, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_p_full + 8 * (t & 1));
+      ok = group_sync();  // T and fin_* are rewritten by the next tile
+      if (!ok) break;
+    }
+    if (ok && n_tiles > 0) {
+      ok = mbar_wait(bar_pv_done + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, 28);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      if (part == 0) {
+        fin_l[col] = l_run;
+        if (col < p.R)
+          p.lse_part[(long long)split * p.rows_total + row0 + col] =
+              (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      }
+      ok = group_sync();
+    }
+    if (ok) {
+      tc_fence_after();
+      float inv[32];
+#pragma unroll
+      for (int n = 0; n < 32; ++n) {
+        const float ln = (n < NP) ? fin_l[n] : 0.f;
+        inv[n] = (ln > 0.f) ? 1.f / ln : 0.f;
+      }
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float o[32];
+        if (n_tiles > 0) {
+          tmem_ld_np<NP>(tw + C::O_COL + nb * NP, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int n = 0; n < 32; ++n) o[n] = 0.f;
+        }
+        const int c = 128 * nb + 32 * warp + lane;  // dv column = TMEM lane of the block
+#pragma unroll
+        for (int n = 0; n < NP; ++n)
+          if (n < p.R) p.o_part[((long long)split * p.rows_total + row0 + n) * p.dv + c] = o[n] * inv[n];
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

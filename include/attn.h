@@ -1,0 +1,161 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so: exact scaled-dot-product attention on NVIDIA B200
+ * (sm_100a).
+ *
+ *   O = softmax(scale * Q.K^T [+ causal mask]) . V,   LSE = ln sum_j exp(scale * q_i.k_j)
+ *
+ * The operation is the standard attention flow S = Q.K^T, P = softmax(S), O = P.V of the
+ * FlashMLA-ETAP technical summary (gist.science 2506.01969, section "Mecanismo Central",
+ * item 1). It is computed tile by tile in on-chip memory with a running-max / running-sum
+ * softmax, so S and P never reach device memory (the "tiling" approach described in
+ * "Activar Flash Attention con llama.cpp", section "Que es Flash Attention"). Key/value heads
+ * may be shared by groups of query heads (GQA; same page, FAQ on GQA).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named q, k, v, o, lse, o_part, lse_part, workspace are DEVICE pointers owned by
+ *    the caller. The library allocates no device memory, never synchronises, and returns as
+ *    soon as the work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream).
+ *  - Layouts are row-major and contiguous:
+ *        q   [B, Hq,  Lq, d]   bf16
+ *        k   [B, Hkv, Lk, d]   bf16
+ *        v   [B, Hkv, Lk, ldv] bf16, the first dv columns of each row are used
+ *        o   [B, Hq,  Lq, dv]  bf16
+ *        lse [B, Hq,  Lq]      fp32 (may be NULL)
+ *  - GQA: query head h reads kv head h / (Hq / Hkv); Hq must be a multiple of Hkv.
+ *  - Causal masking is bottom-right aligned: key j is visible to query row i iff
+ *    j <= i + (Lk - Lq), i.e. the Lq queries are the last Lq positions of the sequence.
+ *    causal != 0 with Lq > Lk is rejected (some rows would see no key).
+ *  - LSE is the natural logarithm of sum_j exp(scale * q_i . k_j) over the visible keys.
+ *  - Arithmetic: bf16 inputs, fp32 accumulation on the tensor cores, fp32 softmax, P rounded
+ *    to bf16 before P.V, O rounded to bf16 (round-to-nearest-even) at the end.
+ *  - Errors: argument checks run on the host before any launch and return a non-zero status
+ *    with nothing enqueued. A failed launch returns ATTN_ERR_CUDA. Kernels bound every wait
+ *    on the GPU; a wait that runs out records ATTN_ERR_TIMEOUT in a device-side word that
+ *    attn_check_device() reads (and clears); the kernel then stops early without hanging.
+ *  - Thread safety: entry points keep no host state between calls except a once-per-process
+ *    lookup of the driver's tensor-map encoder; concurrent calls on different streams are safe.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1, /* NULL pointer, non-positive size, Hq % Hkv, causal Lq > Lk */
+    ATTN_ERR_UNSUPPORTED = 2, /* valid attention, but a shape this build has no kernel for   */
+    ATTN_ERR_MISALIGNED = 3,  /* a pointer or row stride breaks the 16-byte rule of TMA      */
+    ATTN_ERR_WORKSPACE = 4,   /* decode workspace NULL or smaller than required             */
+    ATTN_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed                        */
+    ATTN_ERR_TIMEOUT = 6      /* a bounded wait inside a kernel ran out (see check_device)  */
+} attn_status;
+
+/*
+ * attn_fwd -- prefill / general forward attention.
+ *
+ * Computes O and (optionally) LSE for all B*Hq*Lq query rows against Lk keys. V is dense:
+ * its row stride equals dv.
+ *   scale   multiplies Q.K^T (usually 1/sqrt(d)); must be finite and > 0.
+ *   causal  0 = full attention, non-zero = bottom-right causal mask.
+ * Supported: d == dv, d in {64, 128}; any B, Hq, Hkv (Hq % Hkv == 0), Lq, Lk >= 1.
+ * Kernel: warp-specialised tcgen05/TMEM kernel with TMA loads (one CTA per 128-row Q tile).
+ * Alignment: q, k, v, o 16-byte aligned (row strides are multiples of 16 bytes by shape).
+ */
+attn_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                     int Hq, int Hkv, int Lq, int Lk, int d, int dv, float scale, int causal,
+                     void *stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of device workspace attn_decode needs for the given
+ * shape and split count (num_splits = 0: the count attn_decode chooses on this device).
+ * Layout of the workspace: o_part fp32 [num_splits, B*Hq*Lq, dv] followed (256-byte
+ * aligned) by lse_part fp32 [num_splits, B*Hq*Lq]. Returns 0 for invalid sizes.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv,
+                                  int num_splits);
+
+/*
+ * attn_decode -- split-KV decode attention for a few query tokens against a long KV cache.
+ *
+ * The Lk keys of every (batch, kv head) are cut into num_splits contiguous chunks processed
+ * by different CTAs. Each chunk writes a partial O (fp32, already divided by its own softmax
+ * sum) and a partial LSE (-inf for a chunk without visible keys) into the workspace; an
+ * attn_combine launch on the same stream then merges them into O (bf16) and LSE (fp32).
+ *
+ *   v, ldv   V rows with stride ldv >= dv. MLA latent KV passes v == k and ldv == d: V is the
+ *            first dv columns of each latent K row, and every row is read from memory once.
+ *   num_splits  0 = chosen from the shape and the SM count; otherwise 1..256.
+ *   workspace   device buffer of at least attn_decode_workspace_size(...) bytes, 256-byte
+ *               aligned. Its contents on entry do not matter.
+ * Supported: rows per kv head R = (Hq/Hkv)*Lq <= 64; d <= 576, dv <= 512, d and dv
+ * multiples of 8 (16-byte rows). The tensor-core kernel (key length on the MMA M dimension,
+ * the transposed flow of the FlashMLA-ETAP summary, "Mecanismo Central", items 1-2) serves
+ * d % 64 == 0, dv % 128 == 0, ldv == d when v == k; other shapes use a CUDA-core kernel.
+ */
+attn_status attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+                        int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
+                        float scale, int causal, int num_splits, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
+/* Decode kernels selectable through attn_decode_ex (attn_decode uses ATTN_DECODE_AUTO). */
+typedef enum {
+    ATTN_DECODE_AUTO = 0,      /* tensor-core kernel when the shape allows it, else CUDA cores */
+    ATTN_DECODE_CUDA_CORE = 1, /* fp32 FMA dot products, any supported shape                   */
+    ATTN_DECODE_TCGEN05_T = 2  /* tcgen05, key length on M (transposed flow)                   */
+} attn_decode_impl;
+
+/* attn_decode with an explicit kernel choice (for measurement); ATTN_ERR_UNSUPPORTED if the
+ * requested kernel cannot run the shape. Other arguments as attn_decode. */
+attn_status attn_decode_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                           int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
+                           float scale, int causal, int num_splits, void *workspace,
+                           size_t workspace_bytes, int impl, void *stream);
+
+/*
+ * attn_combine -- log-sum-exp merge of split partials over disjoint key ranges:
+ *   LSE = ln sum_s exp(lse_s),  O = sum_s exp(lse_s - LSE) * O_s   (splits with lse_s = -inf
+ *   carry no weight). o_part fp32 [num_splits, rows, dv], lse_part fp32 [num_splits, rows],
+ *   rows = B*Hq*Lq in [B, Hq, Lq] order; o bf16 [rows, dv]; lse fp32 [rows] (may be NULL).
+ * A row whose every split is empty gets O = 0 and LSE = -inf.
+ */
+attn_status attn_combine(const float *o_part, const float *lse_part, void *o, float *lse,
+                         int B, int Hq, int Lq, int dv, int num_splits, void *stream);
+
+/* Number of splits attn_decode would choose (num_splits = 0) on the current device. */
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv);
+
+/*
+ * attn_check_device -- synchronises `stream`, then reads and clears the device-side error
+ * word that kernels set when a bounded wait runs out. Returns ATTN_OK, ATTN_ERR_TIMEOUT or
+ * ATTN_ERR_CUDA (a sticky CUDA error from earlier work). For tests and diagnostics; the
+ * compute entry points never synchronise.
+ */
+attn_status attn_check_device(void *stream);
+
+/*
+ * attn_selftest_wait_timeout -- diagnostic: launches one CTA that waits on a shared-memory
+ * barrier nothing ever arrives on, with a wall-clock limit of `limit_us` microseconds
+ * (1..1000000). The wait runs out, the kernel records ATTN_ERR_TIMEOUT in the device error word
+ * and returns; the CUDA context stays usable. Pair with attn_check_device() to observe the
+ * status. Enqueued on `stream`; returns ATTN_ERR_INVALID_ARG for a limit outside the range.
+ */
+attn_status attn_selftest_wait_timeout(unsigned int limit_us, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *attn_status_string(attn_status status);
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,151 @@
+"""C ABI checks that need no GPU: the library builds, loads, exports every function declared in
+include/attn.h, and rejects bad arguments on the host before anything is launched.
+
+Pointers passed here are fake addresses (never dereferenced: every call below returns from its
+host-side argument checks).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_139_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA, TIMEOUT = range(7)
+A = 0x10000  # 256-byte aligned fake device address
+B_ = 0x20000
+C_ = 0x30000
+D_ = 0x40000
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build.build()
+    L = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.attn_fwd.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp]
+    L.attn_decode_ex.argtypes = [vp] * 5 + [i] * 8 + [f, i, i, vp, sz, i, vp]
+    L.attn_decode.argtypes = [vp] * 5 + [i] * 8 + [f, i, i, vp, sz, vp]
+    L.attn_combine.argtypes = [vp] * 4 + [i] * 5 + [vp]
+    L.attn_decode_workspace_size.argtypes = [i] * 7
+    L.attn_decode_workspace_size.restype = sz
+    L.attn_status_string.argtypes = [i]
+    L.attn_status_string.restype = ctypes.c_char_p
+    L.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    return L
+
+
+def test_header_declares_expected_entry_points():
+    names = header_functions()
+    for required in ("attn_fwd", "attn_decode", "attn_combine", "attn_decode_workspace_size",
+                     "attn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_header_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+
+
+def test_status_strings(lib):
+    seen = set()
+    for code in range(7):
+        s = lib.attn_status_string(code).decode()
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 7
+    assert lib.attn_status_string(99).decode() == "unknown status"
+    assert lib.attn_abi_version() == 10000
+
+
+def fwd(lib, q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128, scale=0.1,
+        causal=1):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal, None)
+
+
+def test_fwd_argument_checks(lib):
+    assert fwd(lib, q=None) == INVALID
+    assert fwd(lib, o=None) == INVALID
+    assert fwd(lib, B=0) == INVALID
+    assert fwd(lib, Lk=0) == INVALID
+    assert fwd(lib, Hq=3, Hkv=2) == INVALID
+    assert fwd(lib, Lq=256, Lk=128, causal=1) == INVALID
+    assert fwd(lib, scale=0.0) == INVALID
+    assert fwd(lib, scale=float("nan")) == INVALID
+    assert fwd(lib, scale=float("inf")) == INVALID
+    assert fwd(lib, scale=-1.0) == INVALID
+    assert fwd(lib, d=96, dv=96) == UNSUPPORTED
+    assert fwd(lib, d=128, dv=64) == UNSUPPORTED
+    assert fwd(lib, q=A + 8) == MISALIGNED
+    assert fwd(lib, o=D_ + 2) == MISALIGNED
+    assert fwd(lib, lse=A + 2) == MISALIGNED
+
+
+def dec(lib, q=A, k=B_, v=B_, o=D_, lse=None, B=2, Hq=16, Hkv=1, Lq=2, Lk=1000, d=576, dv=512, ldv=576,
+        scale=0.04, causal=1, splits=4, ws=0x100000, ws_bytes=1 << 30, impl=0):
+    return lib.attn_decode_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, splits, ws,
+                              ws_bytes, impl, None)
+
+
+def test_decode_argument_checks(lib):
+    assert dec(lib, q=None) == INVALID
+    assert dec(lib, Hq=15, Hkv=2) == INVALID
+    assert dec(lib, ldv=256) == INVALID           # ldv < dv
+    assert dec(lib, splits=-1) == INVALID
+    assert dec(lib, splits=257) == INVALID
+    assert dec(lib, impl=7) == INVALID
+    assert dec(lib, Lq=3, Lk=2) == INVALID         # causal with Lq > Lk
+    assert dec(lib, d=100, dv=96, ldv=100) == MISALIGNED  # 200-byte rows are not 16-byte multiples
+    assert dec(lib, Hq=64, Lq=2) == UNSUPPORTED    # 128 rows per kv head
+    assert dec(lib, d=640, dv=512, ldv=640) == UNSUPPORTED
+    assert dec(lib, v=C_, ldv=512, impl=2) == UNSUPPORTED  # tensor-core kernel needs latent KV
+    assert dec(lib, ws=None) == WORKSPACE
+    assert dec(lib, ws_bytes=1024) == WORKSPACE
+    assert dec(lib, ws=0x100010) == WORKSPACE      # not 256-byte aligned
+    assert dec(lib, k=B_ + 4, v=B_ + 4) == MISALIGNED
+
+
+def test_combine_argument_checks(lib):
+    f = lambda **kw: lib.attn_combine(kw.get("op", A), kw.get("lp", B_), kw.get("o", C_), kw.get("lse", None),
+                                      kw.get("B", 1), kw.get("Hq", 2), kw.get("Lq", 3), kw.get("dv", 64),
+                                      kw.get("S", 4), None)
+    assert f(op=None) == INVALID
+    assert f(o=None) == INVALID
+    assert f(S=0) == INVALID
+    assert f(dv=62) == MISALIGNED
+    assert f(op=A + 4) == MISALIGNED
+
+
+def test_workspace_size_formula(lib):
+    def ref(B, Hq, Lq, dv, s):
+        a = lambda x: (x + 255) // 256 * 256
+        rows = B * Hq * Lq
+        return a(s * rows * dv * 4) + a(s * rows * 4)
+    for args in [(32, 16, 1, 2, 65536, 512, 9), (1, 1, 1, 1, 1, 8, 1), (4, 8, 2, 1, 5000, 128, 37)]:
+        B, Hq, Hkv, Lq, Lk, dv, s = args
+        assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, s) == ref(B, Hq, Lq, dv, s)
+    assert lib.attn_decode_workspace_size(0, 1, 1, 1, 1, 8, 1) == 0
+    assert lib.attn_decode_workspace_size(1, 3, 2, 1, 1, 8, 1) == 0
+    assert lib.attn_decode_workspace_size(1, 1, 1, 1, 1, 8, 300) == 0
+
+
+def test_selftest_limit_checked(lib):
+    assert lib.attn_selftest_wait_timeout(0, None) == INVALID
+    assert lib.attn_selftest_wait_timeout(2_000_000, None) == INVALID
+
+
+def test_binding_has_c_names():
+    from exact_attention_139_b200 import attn
+    for name in ("attn_fwd", "attn_decode", "attn_combine", "attn_decode_workspace_size", "attn_status_string",
+                 "attn_check_device"):
+        assert callable(getattr(attn, name))
