@@ -1,0 +1,383 @@
+"""Benchmark: exact attention on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the hot path over one batch of synthetic input. The default workload is the
+Llama-3-8B-shaped causal GQA prefill (B=1, Hq=32, Hkv=8, L=8192, d=128): metric attention TFLOPS
+(algorithmic flops = 2*(d+dv) per visible query/key pair). The same JSON line also carries the
+MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) measured in
+HBM GB/s, each with its roofline fraction against MEASURED_PEAKS.json.
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching stream;
+L2 is flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU (torchrun):
+every rank runs its own copy of the workload (independent batches: weak scaling, no collective on
+the data path); the per-rank time is max-reduced and value = total flops of all ranks / max time.
+
+--impl reference times the fp64 CPU oracle on a bounded seeded sample of the same workload (the
+reference arm: the pages ship no runnable code, so the oracle is the reference program).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from exact_attention_139_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU every ~10 ms from a
+    background thread through NVML (read-only queries), during the timed region."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.thread = None
+
+    def _run(self):
+        import pynvml
+        try:
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self.stop_flag:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                try:
+                    reasons = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except AttributeError:
+                    reasons = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                self.samples.append((sm, reasons))
+                time.sleep(0.01)
+        except Exception as e:  # clocks are reported as unavailable, the run itself continues
+            self.error = str(e)
+
+    def start(self):
+        import threading
+        self.stop_flag = False
+        self.error = None
+        self.max_mhz = None
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        time.sleep(0.05)
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return {"error": self.error} if self.error else None
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# timing helpers
+# ------------------------------------------------------------------------------------------------
+class Flusher:
+    def __init__(self, dev):
+        self.buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_steps(step, steps, warmup, flush, stream):
+    """Per-step CUDA-event durations (ms) of `step` on `stream`, L2 flushed before each step."""
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """Max of a per-rank scalar over the process group (the slowest rank sets the job time)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Each rank processes its own independent batch (same shape, its own seed)."""
+    return w if rank == 0 else w.with_(seed=w.seed + 1000 * rank)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU baseline / reference arm: the fp64 oracle on a bounded sample
+# ------------------------------------------------------------------------------------------------
+def oracle_sample_rate(w, target_s: float, q=None, k=None, v=None):
+    """Time the oracle on seeded rows of workload w; returns (flops/s, rows, seconds, threads)."""
+    from oracle import oracle
+    if q is None:
+        q, k, v = make_inputs(w)
+    g = np.random.default_rng(12345)
+    threads = oracle.default_threads()
+    # calibrate on a small batch, then size the sample to ~target_s seconds
+    n = 64
+    total_rows = w.B * w.Hq * w.Lq
+    while True:
+        rows = np.sort(g.choice(total_rows, size=min(n, total_rows), replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_rows(q, k, (k if w.latent else v), rows, B=w.B, Hq=w.Hq, Hkv=w.Hkv, Lq=w.Lq, Lk=w.Lk, d=w.d,
+                         dv=w.dv, ldv=w.ldv, scale=w.scale, causal=w.causal, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n >= total_rows:
+            break
+        n = int(min(total_rows, max(2 * n, n * target_s / max(dt, 1e-3) * 1.05)))
+    flops = 0.0
+    off = w.Lk - w.Lq
+    for r in rows:
+        i = int(r) % w.Lq
+        vis = min(w.Lk, i + off + 1) if w.causal else w.Lk
+        flops += vis * 2.0 * (w.d + w.dv)
+    return flops / dt, len(rows), dt, threads
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+def bench_prefill(w, dev, steps, warmup, flush, stream):
+    from exact_attention_139_b200 import attn
+    q, k, v = make_inputs(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    step = lambda: attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    times = time_steps(step, steps, warmup, flush, stream)
+    if attn.attn_check_device() != attn.ATTN_OK:
+        raise RuntimeError("device error during the prefill benchmark")
+    return times, (q, k, v)
+
+
+def bench_prefill_e2e(w, dev, steps, warmup, host):
+    """End to end: pinned host inputs -> device, attn_fwd, O and LSE back to pinned host memory."""
+    from exact_attention_139_b200 import attn
+    q, k, v = (t.pin_memory() for t in host)
+    bufs = {}
+    for _ in range(max(1, warmup)):
+        attn.attn_fwd_host(q, k, v, causal=w.causal, scale=w.scale, device=dev, bufs=bufs)
+    stream = torch.cuda.current_stream(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        attn.attn_fwd_host(q, k, v, causal=w.causal, scale=w.scale, device=dev, bufs=bufs)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = bufs["o_host"].numel() * 2 + bufs["lse_host"].numel() * 4
+    return ms, h2d, d2h
+
+
+def bench_decode(w, dev, steps, warmup, flush, stream):
+    from exact_attention_139_b200 import attn
+    q, k, _ = make_inputs(w)
+    qd, kd = q.to(dev), k.to(dev)
+    del q, k
+    splits = attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv)
+    ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, splits),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    step = lambda: attn.attn_decode(qd, kd, kd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=splits,
+                                    workspace=ws, out=o, lse=lse)
+    times = time_steps(step, steps, warmup, flush, stream)
+    if attn.attn_check_device() != attn.ATTN_OK:
+        raise RuntimeError("device error during the decode benchmark")
+    # time the split kernel alone (the combine is the second launch of each step)
+    return times, splits
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = rank_workload(WORKLOADS[args.workload], rank)
+    stream = torch.cuda.current_stream(dev)
+    flush = Flusher(dev)
+    clocks = ClockSampler(torch.cuda.current_device())
+
+    barrier(world)
+    clocks.start()
+    times, host = bench_prefill(w, dev, args.steps, args.warmup, flush, stream)
+    clk = clocks.stop()
+    barrier(world)
+    ms_local = sum(times) / len(times)
+    ms = max_over_ranks(ms_local, world)
+    flops = w.flops()
+    value = flops * world / (ms * 1e-3) / 1e12
+    per_gpu_tflops = flops / (ms * 1e-3) / 1e12
+    peak_tf = float(peaks["bf16_tflops"])
+
+    extras = {}
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = bench_prefill_e2e(w, dev, max(2, args.steps // 2), 1, host)
+        e_ms = max_over_ranks(e_ms, world)
+        e2e = {"value": round(flops * world / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
+    del host
+    launches = args.steps  # one prefill kernel per step
+    if not args.no_extras:
+        wd = rank_workload(WORKLOADS["mla_decode_64k"], rank)
+        clocks_d = ClockSampler(torch.cuda.current_device())
+        clocks_d.start()
+        dtimes, splits = bench_decode(wd, dev, args.steps, args.warmup, flush, stream)
+        dclk = clocks_d.stop()
+        dms = max_over_ranks(sum(dtimes) / len(dtimes), world)
+        gbs = wd.kv_bytes() / (dms * 1e-3) / 1e9
+        extras["decode"] = {
+            "workload": wd.name, "metric": "KV-read HBM GB/s", "value": round(gbs * world, 1),
+            "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits,
+            "kernels_per_step": 2,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": wd.kv_bytes(), "traffic": None,
+                         "note": "step = split kernel + combine kernel"},
+            "tflops": round(wd.flops() / (dms * 1e-3) / 1e12, 1), "clocks": dclk}
+        launches += 2 * args.steps
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, nrows, secs, threads = oracle_sample_rate(w, args.cpu_seconds)
+        cpu = {"value": round(rate / 1e12, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+               "sample": f"{nrows} seeded query rows of {w.name} (fp64 oracle, {secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": "attention TFLOPS (causal GQA prefill, Llama-3-8B shape)" if w.causal else "attention TFLOPS",
+            "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+                       "dv": w.dv, "causal": w.causal, "flops_per_step_per_gpu": flops,
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(per_gpu_tflops / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "algorithmic_flops_per_launch": flops, "traffic": None},
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    q, k, v = make_inputs(w)
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, min(2.0, args.cpu_seconds / 4), q, k, v)
+    rows_used, threads = 0, 1
+    for _ in range(args.steps):
+        rate, rows_used, secs, threads = oracle_sample_rate(w, args.cpu_seconds / max(1, args.steps), q, k, v)
+        per_step.append(rate)
+    value = statistics.mean(per_step) / 1e12
+    line = {
+        "impl": "reference", "metric": "attention TFLOPS (causal GQA prefill, Llama-3-8B shape)",
+        "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+                   "dv": w.dv, "causal": w.causal},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_used} seeded query rows per step of {w.name} (fp64 oracle)"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_prefill_8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU (oracle) baseline")
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -51,7 +51,7 @@ _lib.attn_abi_version.argtypes = []
 
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED = 0, 1, 2, 3
 ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = 4, 5, 6
-ATTN_DECODE_AUTO, ATTN_DECODE_CUDA_CORE, ATTN_DECODE_TCGEN05_T = 0, 1, 2
+ATTN_DECODE_AUTO, ATTN_DECODE_CUDA_CORE, ATTN_DECODE_TCGEN05_T, ATTN_DECODE_TCGEN05_N = 0, 1, 2, 3
 
 
 class AttnError(RuntimeError):

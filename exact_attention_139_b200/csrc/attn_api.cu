@@ -186,6 +186,39 @@ attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
   }
 }
 
+template <int DCH, int NPIECE>
+attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
+  using C = attn::DecodeTnCfg<DCH, NPIECE>;
+  CUtensorMap tq, tkv;
+  if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
+  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, C::BK)) return ATTN_ERR_CUDA;
+  auto kern = attn::decode_tn_kernel<DCH, NPIECE>;
+  if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  dim3 grid(splits, p.B * p.Hkv);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, p);
+  return launch_status();
+}
+
+template <int DCH>
+attn_status launch_tn_np(const DecodeParams& p, int splits, cudaStream_t st) {
+  if (p.dv <= 256) return launch_tn<DCH, 1>(p, splits, st);
+  return launch_tn<DCH, 2>(p, splits, st);
+}
+
+attn_status launch_tn_any(const DecodeParams& p, int splits, cudaStream_t st) {
+  switch (p.d / 64) {
+    case 2: return launch_tn_np<2>(p, splits, st);
+    case 3: return launch_tn_np<3>(p, splits, st);
+    case 4: return launch_tn_np<4>(p, splits, st);
+    case 5: return launch_tn_np<5>(p, splits, st);
+    case 6: return launch_tn_np<6>(p, splits, st);
+    case 7: return launch_tn_np<7>(p, splits, st);
+    case 8: return launch_tn_np<8>(p, splits, st);
+    case 9: return launch_tn_np<9>(p, splits, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
 attn_status launch_tc_any(const DecodeParams& p, int splits, cudaStream_t st) {
   switch (p.d / 64) {
     case 2: return launch_tc_nb<2>(p, splits, st);
@@ -303,12 +336,13 @@ attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o,
   if (st != ATTN_OK) return st;
   if (ldv < dv) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
-  if (impl < ATTN_DECODE_AUTO || impl > ATTN_DECODE_TCGEN05_T) return ATTN_ERR_INVALID_ARG;
+  if (impl < ATTN_DECODE_AUTO || impl > ATTN_DECODE_TCGEN05_N) return ATTN_ERR_INVALID_ARG;
   if (d % 8 != 0 || dv % 8 != 0 || ldv % 8 != 0) return ATTN_ERR_MISALIGNED;
   const bool tc_ok = tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
   const bool cc_ok = cc_supported(Hq, Hkv, Lq, d, dv, ldv);
-  if (impl == ATTN_DECODE_AUTO) impl = tc_ok ? ATTN_DECODE_TCGEN05_T : ATTN_DECODE_CUDA_CORE;
-  if (impl == ATTN_DECODE_TCGEN05_T && !tc_ok) return ATTN_ERR_UNSUPPORTED;
+  // both tensor-core kernels serve the same shapes (tc_ok)
+  if (impl == ATTN_DECODE_AUTO) impl = tc_ok ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
+  if ((impl == ATTN_DECODE_TCGEN05_T || impl == ATTN_DECODE_TCGEN05_N) && !tc_ok) return ATTN_ERR_UNSUPPORTED;
   if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
   int splits = num_splits;
   if (splits == 0) splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
@@ -341,6 +375,8 @@ attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o,
 
   if (impl == ATTN_DECODE_TCGEN05_T) {
     st = launch_tc_any(p, splits, cs);
+  } else if (impl == ATTN_DECODE_TCGEN05_N) {
+    st = launch_tn_any(p, splits, cs);
   } else {
     const int cpt = (dv + attn::kCcThreads - 1) / attn::kCcThreads;
     if (p.R <= 16) st = cpt == 1 ? launch_cc<16, 1>(p, splits, cs) : launch_cc<16, 2>(p, splits, cs);

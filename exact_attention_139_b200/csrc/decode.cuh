@@ -555,4 +555,294 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
   }
 }
 
+// ======================================================================================
+// tcgen05 kernel, queries on the MMA M dimension (padded to 64), keys on N
+// ======================================================================================
+// S = Q.K^T with M = 64 query rows (R <= 32 real rows; rows 32..63 read whatever follows in
+// shared memory and are never used: MMA rows are independent), N = 64 keys, K = d. Each
+// softmax thread then owns one query row and reduces over its keys in registers, so a tile
+// needs no block-level synchronisation. O = P.V with M = 64, N = dv in pieces of <= 256.
+// TMEM (M = 64 layout: row m lives in lane (m % 16) + 32 * (m / 16) of a half):
+//   lane half 0 (lanes 0-15 of each quadrant): O, columns [0, dv)
+//   lane half 1 (lanes 16-31 of each quadrant): S double buffer, columns [0, 64) and [64, 128)
+// Warps: 0-1 softmax (lanes 16-31 hold S rows, lanes 0-15 the matching O rows), 2 TMA producer,
+// 3 TMEM allocator + MMA issuer.
+template <int DCH, int NPIECE>
+struct DecodeTnCfg {
+  static constexpr int BK = 64;                  // keys per tile (MMA N of S)
+  static constexpr int KCH = BK * 128;           // one 64-key x 128-byte chunk
+  static constexpr int STAGE = DCH * KCH;
+  static constexpr int QCH = 32 * 128;           // 32 query rows x 128 bytes
+  static constexpr int PB = 32 * 128;            // P tile: 32 rows x 64 keys bf16
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_Q = OFF_KV + 2 * STAGE;
+  static constexpr int OFF_P = OFF_Q + DCH * QCH;   // right after Q: rows 32..63 of the M=64 reads
+  static constexpr int OFF_PAD = OFF_P + 2 * PB;    // 4 KB of slack read as rows 32..63 of P1
+  static constexpr int OFF_BAR = OFF_PAD + 4096;
+  // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int N_BARS = 12;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
+  static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t S_LANE = 16;
+  static constexpr int THREADS = 128;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int DCH, int NPIECE>
+__global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
+    decode_tn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                     const DecodeParams p) {
+  using C = DecodeTnCfg<DCH, NPIECE>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int split = blockIdx.x;
+  const int unit = blockIdx.y;
+  const int b = unit / p.Hkv, hkv = unit % p.Hkv;
+  const long long row0 = ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
+  const int j_begin = split * p.chunk;
+  const int j_end = min(p.Lk, j_begin + p.chunk);
+  const int n_tiles = j_end > j_begin ? (j_end - j_begin + C::BK - 1) / C::BK : 0;
+  const int off = p.Lk - p.Lq;
+  const int NW = p.dv / NPIECE;  // columns per O piece (multiple of 64)
+  const uint32_t TMEM_COLS = p.dv <= 128 ? 128u : (p.dv <= 256 ? 256u : 512u);
+
+  const uint32_t bar_q = base + C::OFF_BAR;
+  const uint32_t bar_kv_full = bar_q + 8;
+  const uint32_t bar_kv_empty = bar_kv_full + 16;
+  const uint32_t bar_s_full = bar_kv_empty + 16;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_pv_done = bar_p_full + 16;
+  const uint32_t bar_drain = bar_pv_done + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_kv_full + 8 * i, 1);
+      mbar_init(bar_kv_empty + 8 * i, 1);
+      mbar_init(bar_s_full + 8 * i, 1);
+      mbar_init(bar_p_full + 8 * i, 64);
+      mbar_init(bar_pv_done + 8 * i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 3) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 2) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kv);
+      mbar_arrive_expect_tx(bar_q, DCH * C::QCH);
+#pragma unroll
+      for (int c = 0; c < DCH; ++c) tma_load_2d(base + C::OFF_Q + c * C::QCH, &tm_q, bar_q, 64 * c, (int)row0);
+      const int z = b * p.Hkv + hkv;
+      int t = 0;
+      bool ok = true;
+      for (; t < n_tiles; ++t) {
+        const int s = t & 1;
+        if (t >= 2) ok = mbar_wait(bar_kv_empty + 8 * s, ((t >> 1) & 1) ^ 1, 41);
+        if (!ok) break;
+        const uint32_t full = bar_kv_full + 8 * s;
+        mbar_arrive_expect_tx(full, C::STAGE);
+#pragma unroll
+        for (int c = 0; c < DCH; ++c)
+          tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * C::BK, z);
+      }
+      if (!ok) {
+        mbar_wait_drain(bar_q, 0);
+        for (int u = max(0, t - 2); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u & 1), (u >> 1) & 1);
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(64, C::BK, false, false);  // S = Q.K^T
+      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);         // O += P.V
+      const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL;
+      bool ok = mbar_wait(bar_q, 0, 42);
+      bool issued = false;
+      auto pv = [&](int tt) {
+        ok = mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 43);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KV + (tt & 1) * C::STAGE;
+        const uint32_t pb = base + C::OFF_P + (tt & 1) * C::PB;
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk) {
+          const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
+#pragma unroll
+          for (int h = 0; h < NPIECE; ++h) {
+            // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
+            const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
+            mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_kv_empty + 8 * (tt & 1));
+        mma_commit(bar_pv_done + 8 * (tt & 1));
+      };
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        ok = mbar_wait(bar_kv_full + 8 * (t & 1), (t >> 1) & 1, 44);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KV + (t & 1) * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < 4 * DCH; ++kk) {
+          const uint64_t ad = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          mma_ss(s_tmem + (t & 1) * C::BK, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        mma_commit(bar_s_full + 8 * (t & 1));
+        if (t > 0) pv(t - 1);
+      }
+      if (ok) pv(n_tiles - 1);
+      if (!ok && issued) {
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else {
+    // --------------------------- softmax warps 0-1 ---------------------------
+    const bool s_lane = lane >= 16;
+    const int m = 16 * warp + (lane & 15);  // query row (S row for lanes 16-31, O row for 0-15)
+    const bool row_ok = m < p.R;
+    const int qi = m % p.Lq;
+    const uint32_t tw = tmem + ((uint32_t)(warp * 32) << 16);
+    const float c2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      ok = mbar_wait(bar_s_full + 8 * (t & 1), (t >> 1) & 1, 45);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float x[2][32];
+      tmem_ld32(tw + C::S_COL + (t & 1) * C::BK, x[0]);
+      tmem_ld32(tw + C::S_COL + (t & 1) * C::BK + 32, x[1]);
+      tmem_wait_ld();
+      const int k0 = j_begin + t * C::BK;
+      int lim = j_end - 1;
+      if (p.causal) lim = min(lim, qi + off);
+      const int rem = lim - k0;  // keys c <= rem of this tile are visible
+      float mx = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (32 * h + e > rem) x[h][e] = -INFINITY;
+          mx = fmaxf(mx, x[h][e]);
+        }
+      const float m_tile = mx * c2;
+      float alpha = 1.f;
+      if (m_tile != -INFINITY) {
+        if (m_run == -INFINITY) {
+          m_run = m_tile;  // O row and l are still zero: nothing to rescale
+        } else if (m_tile > m_run + kRescaleLog2) {
+          alpha = ex2_approx(m_run - m_tile);
+          m_run = m_tile;
+        }
+      }
+      const float m_ref = (m_run == -INFINITY) ? 0.f : m_run;
+      // P buffer (t & 1) is free once P.V of tile t-2 has completed
+      if (t >= 2) {
+        ok = mbar_wait(bar_pv_done + 8 * (t & 1), ((t - 2) >> 1) & 1, 46);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      float sum = 0.f;
+      uint8_t* prow = smem + C::OFF_P + (t & 1) * C::PB;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // 8 keys per 16-byte unit
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v0 = x[u >> 2][(8 * u + 2 * e) & 31];
+          const float v1 = x[u >> 2][(8 * u + 2 * e + 1) & 31];
+          const float p0 = ex2_approx(fmaf(v0, c2, -m_ref));
+          const float p1 = ex2_approx(fmaf(v1, c2, -m_ref));
+          sum += p0 + p1;
+          w4[e] = pack_bf16x2(p0, p1);
+        }
+        if (s_lane)
+          *reinterpret_cast<uint4*>(prow + swz128_offset((uint32_t)m, (uint32_t)u)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      l_run = l_run * alpha + sum;
+      // rescale the O rows whose reference moved (rare): lanes 0-15 own those O rows
+      const float alpha_o = __shfl_down_sync(0xffffffffu, alpha, 16);
+      const bool need = t > 0 && __any_sync(0xffffffffu, s_lane && alpha != 1.f);
+      if (need) {
+        // O is stable once P.V of tile t-1 is done; S of tile t+1 (same columns, other lane
+        // half, rewritten unchanged below) must have landed too
+        ok = mbar_wait(bar_pv_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, 47);
+        if (ok && t + 1 < n_tiles) ok = mbar_wait(bar_s_full + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, 48);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float a = s_lane ? 1.f : alpha_o;
+        for (int cg = 0; cg < p.dv / 32; ++cg) {
+          float o[32];
+          tmem_ld32(tw + 32 * cg, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= a;
+          tmem_st32(tw + 32 * cg, o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_p_full + 8 * (t & 1));
+    }
+    if (ok && n_tiles > 0) {
+      ok = mbar_wait(bar_pv_done + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, 49);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      // lanes 16-31 hold (m_run, l_run) of row m; lanes 0-15 hold O row m
+      const float l_o = __shfl_down_sync(0xffffffffu, l_run, 16);
+      if (s_lane && row_ok)
+        p.lse_part[(long long)split * p.rows_total + row0 + m] =
+            (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      const float inv = (l_o > 0.f) ? 1.f / l_o : 0.f;
+      float* dst = p.o_part + ((long long)split * p.rows_total + row0 + m) * p.dv;
+      tc_fence_after();
+      for (int cg = 0; cg < p.dv / 32; ++cg) {
+        float o[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tw + 32 * cg, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (!s_lane && row_ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * cg + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 3) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 }  // namespace attn

@@ -95,9 +95,11 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv
  *   workspace   device buffer of at least attn_decode_workspace_size(...) bytes, 256-byte
  *               aligned. Its contents on entry do not matter.
  * Supported: rows per kv head R = (Hq/Hkv)*Lq <= 64; d <= 576, dv <= 512, d and dv
- * multiples of 8 (16-byte rows). The tensor-core kernel (key length on the MMA M dimension,
- * the transposed flow of the FlashMLA-ETAP summary, "Mecanismo Central", items 1-2) serves
- * d % 64 == 0, dv % 128 == 0, ldv == d when v == k; other shapes use a CUDA-core kernel.
+ * multiples of 8 (16-byte rows). Two tensor-core kernels serve latent KV (v == k, ldv == d)
+ * with d % 64 == 0, dv % 128 == 0, dv <= d and R <= 32: one puts the key length on the MMA M
+ * dimension (the transposed flow of the FlashMLA-ETAP summary, "Mecanismo Central", items 1-3),
+ * the other puts the query rows on M (padded to 64) and keys on N; attn_decode uses the one
+ * measured faster on B200. Other shapes use a CUDA-core kernel.
  */
 attn_status attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
                         int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
@@ -108,7 +110,8 @@ attn_status attn_decode(const void *q, const void *k, const void *v, void *o, fl
 typedef enum {
     ATTN_DECODE_AUTO = 0,      /* tensor-core kernel when the shape allows it, else CUDA cores */
     ATTN_DECODE_CUDA_CORE = 1, /* fp32 FMA dot products, any supported shape                   */
-    ATTN_DECODE_TCGEN05_T = 2  /* tcgen05, key length on M (transposed flow)                   */
+    ATTN_DECODE_TCGEN05_T = 2, /* tcgen05, key length on M (transposed flow)                   */
+    ATTN_DECODE_TCGEN05_N = 3  /* tcgen05, query rows on M (padded to 64), keys on N            */
 } attn_decode_impl;
 
 /* attn_decode with an explicit kernel choice (for measurement); ATTN_ERR_UNSUPPORTED if the

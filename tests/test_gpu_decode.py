@@ -9,7 +9,7 @@ from tests.gpu_util import compare, oracle_rows, rows_per_head, take_rows
 
 pytestmark = pytest.mark.gpu
 
-CC, TC = 1, 2
+CC, TC, TN = 1, 2, 3
 
 
 def run(w, dev, impl=0, num_splits=0):
@@ -23,12 +23,12 @@ def run(w, dev, impl=0, num_splits=0):
     return q, k, v, o, lse
 
 
-@pytest.mark.parametrize("impl", [TC, CC])
+@pytest.mark.parametrize("impl", [TN, TC, CC])
 def test_mla_decode_64k(impl, cuda_device):
     w = WORKLOADS["mla_decode_64k"]
     q, k, v, o, lse = run(w, cuda_device, impl=impl)
-    # every row of the first batches (rows_per_head * Hq rows in all)
-    nb = max(1, rows_per_head(2) // 2)
+    # every row of the first nb batches (all 32 batches by default: the full output)
+    nb = min(w.B, max(1, rows_per_head(2 * w.B) // 2))
     rows = np.arange(nb * w.Hq * w.Lq)
     o_ref, l_ref = oracle_rows(w, q, k, v, rows)
     og, lg = take_rows(o, lse, rows)
@@ -59,7 +59,7 @@ def test_small_shapes(shape, splits, cuda_device):
     o_ref, l_ref = oracle_rows(w, q, k, v, rows)
     impls = [CC]
     if latent and d % 64 == 0 and dv % 128 == 0 and (Hq // Hkv) * Lq <= 32:
-        impls.append(TC)
+        impls += [TC, TN]
     qd, kd = q.to(cuda_device), k.to(cuda_device)
     vd = kd if latent else v.to(cuda_device)
     for impl in impls:
@@ -71,7 +71,7 @@ def test_small_shapes(shape, splits, cuda_device):
 def test_split_count_invariance(cuda_device):
     from exact_attention_139_b200 import attn
     w = Workload("inv", 2, 16, 1, 2, 5000, 576, 512, True, latent=True, seed=31)
-    q, k, _ = (t.to(cuda_device) if t is not None else None for t in make_inputs(w))
+    q, k, _ = (t.to(cuda_device) for t in make_inputs(w))
     outs = [attn.attn_decode(q, k, k, causal=True, dv=512, num_splits=s)[0].float() for s in (1, 5, 40)]
     for o in outs[1:]:
         assert (o - outs[0]).abs().max().item() <= 1e-2
