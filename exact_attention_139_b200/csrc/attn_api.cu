@@ -394,6 +394,56 @@ attn_status attn_decode(const void* q, const void* k, const void* v, void* o, fl
                         ws_bytes, ATTN_DECODE_AUTO, stream);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Allocation-free decode: split partials live in a scratch array compiled into the library.
+// ---------------------------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+// The scratch array. In host code its name is only a stand-in for the symbol; kernels must be
+// given the device address looked up below.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+attn_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                                int Hkv, int Lq, int Lk, int d, int dv, int ldv, float scale, int causal,
+                                int num_splits, void* stream) {
+  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
+  const int splits = num_splits > 0 ? num_splits : choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  const size_t need = workspace_bytes((long long)B * Hq * Lq, dv, splits);
+  if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != ATTN_OK) return st;
+  return attn_decode_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, splits, scratch,
+                        (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES, ATTN_DECODE_AUTO, stream);
+}
+
 attn_status attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq, int Lq,
                          int dv, int num_splits, void* stream) {
   if (!o_part || !lse_part || !o) return ATTN_ERR_INVALID_ARG;

@@ -122,6 +122,33 @@ attn_status attn_decode_ex(const void *q, const void *k, const void *v, void *o,
                            size_t workspace_bytes, int impl, void *stream);
 
 /*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
+ *
+ * No counterpart in the pages; this is an interface addition. Some callers cannot call
+ * cudaMalloc or hand over a workspace: code that runs while a CUDA graph is being captured
+ * elsewhere in the process, memory-capped serving processes with a fixed pool, or plugins that
+ * only receive input and output pointers. This entry point takes the same arguments as
+ * attn_decode minus the workspace and keeps the split partials in a scratch array compiled
+ * into the library: ATTN_DECODE_NOALLOC_SCRATCH_BYTES bytes of device memory that every GPU
+ * which loads the library holds until the process exits. It calls no allocating routine.
+ *   - Shapes whose partials (attn_decode_workspace_size for the chosen split count) exceed
+ *     the scratch size are rejected with ATTN_ERR_WORKSPACE before anything is enqueued; pass a
+ *     smaller num_splits or use attn_decode with a caller workspace.
+ *   - The first call on each device looks up the device address of the scratch array (a
+ *     synchronous host call that may load the library's GPU code). Make that first call before
+ *     any stream capture on that device.
+ *   - All calls share the one array and it keeps the last call's contents. The kernels write
+ *     every scratch byte they later read, so nothing needs clearing between calls, but two
+ *     calls that overlap on the GPU (different streams, no ordering between them) race on the
+ *     array and give wrong results. Order such calls on one stream or with events.
+ * Other arguments, supported shapes and kernel choice are those of attn_decode.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+attn_status attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
+                                float scale, int causal, int num_splits, void *stream);
+
+/*
  * attn_combine -- log-sum-exp merge of split partials over disjoint key ranges:
  *   LSE = ln sum_s exp(lse_s),  O = sum_s exp(lse_s - LSE) * O_s   (splits with lse_s = -inf
  *   carry no weight). o_part fp32 [num_splits, rows, dv], lse_part fp32 [num_splits, rows],
