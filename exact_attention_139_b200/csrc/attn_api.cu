@@ -16,6 +16,7 @@
 #include "combine.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill2.cuh"
 
 namespace {
 
@@ -23,6 +24,12 @@ using attn::DecodeParams;
 using attn::PrefillParams;
 
 constexpr int kAbiVersion = 10000;  // 1.0.0
+
+#ifndef ATTN_PREFILL_VERSION
+#define ATTN_PREFILL_VERSION 2
+#endif
+// 2: persistent two-tile kernel (prefill2.cuh); 1: one 128-row tile per CTA (prefill.cuh).
+constexpr int kPrefillVersion = ATTN_PREFILL_VERSION;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -186,13 +193,22 @@ attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
   }
 }
 
+#ifndef ATTN_TN_BK
+#define ATTN_TN_BK 48
+#endif
+#ifndef ATTN_TN_NST
+#define ATTN_TN_NST 3
+#endif
+// Key tile and stage count of the queries-on-M decode kernel (chosen by measurement on B200).
+constexpr int kTnBK = ATTN_TN_BK, kTnNST = ATTN_TN_NST;
+
 template <int DCH, int NPIECE>
 attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
-  using C = attn::DecodeTnCfg<DCH, NPIECE>;
+  using C = attn::DecodeTnCfg<DCH, NPIECE, kTnBK, kTnNST>;
   CUtensorMap tq, tkv;
   if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
-  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, C::BK)) return ATTN_ERR_CUDA;
-  auto kern = attn::decode_tn_kernel<DCH, NPIECE>;
+  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK)) return ATTN_ERR_CUDA;
+  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, kTnNST>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, p);
@@ -280,6 +296,41 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
   if (st != ATTN_OK) return st;
   if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int n_qtiles = (Lq + 127) / 128;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bf16(&tq, q, (uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
+      !encode_bf16(&tk, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
+      !encode_bf16(&tv, v, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
+    return ATTN_ERR_CUDA;
+  if (kPrefillVersion == 2) {
+    attn::Prefill2Params p{};
+    p.o = reinterpret_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.G = Hq / Hkv;
+    p.n_pairs = (n_qtiles + 1) / 2;
+    const long long units = (long long)p.n_pairs * B * Hq;
+    if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    p.n_units = (int)units;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int grid = (int)std::min<long long>(units, current_sm_count());
+    if (d == 128) {
+      using C = attn::Prefill2Cfg<128>;
+      if (!allow_smem(attn::prefill2_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+      attn::prefill2_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    } else {
+      using C = attn::Prefill2Cfg<64>;
+      if (!allow_smem(attn::prefill2_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+      attn::prefill2_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    }
+    return launch_status();
+  }
   PrefillParams p{};
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -289,27 +340,17 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Lq = Lq;
   p.Lk = Lk;
   p.G = Hq / Hkv;
-  p.n_qtiles = (Lq + 127) / 128;
+  p.n_qtiles = n_qtiles;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = (long long)p.n_qtiles * B * Hq;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  CUtensorMap tq, tk, tv;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (d == 128) {
     using C = attn::PrefillCfg<128>;
-    if (!encode_bf16(&tq, q, 128, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
-        !encode_bf16(&tk, k, 128, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
-        !encode_bf16(&tv, v, 128, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
-      return ATTN_ERR_CUDA;
     if (!allow_smem(attn::prefill_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
     attn::prefill_kernel<128><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   } else {
     using C = attn::PrefillCfg<64>;
-    if (!encode_bf16(&tq, q, 64, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
-        !encode_bf16(&tk, k, 64, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
-        !encode_bf16(&tv, v, 64, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
-      return ATTN_ERR_CUDA;
     if (!allow_smem(attn::prefill_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
     attn::prefill_kernel<64><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   }

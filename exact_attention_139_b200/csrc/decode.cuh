@@ -558,42 +558,70 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
 // ======================================================================================
 // tcgen05 kernel, queries on the MMA M dimension (padded to 64), keys on N
 // ======================================================================================
-// S = Q.K^T with M = 64 query rows (R <= 32 real rows; rows 32..63 read whatever follows in
-// shared memory and are never used: MMA rows are independent), N = 64 keys, K = d. Each
-// softmax thread then owns one query row and reduces over its keys in registers, so a tile
+// S = Q.K^T with M = 64 query rows (R <= 32 real rows; rows 32..63 of the A operand read whatever
+// follows in shared memory and are never used: MMA rows are independent), N = BK keys, K = d.
+// Each softmax thread then owns one query row and reduces over its keys in registers, so a tile
 // needs no block-level synchronisation. O = P.V with M = 64, N = dv in pieces of <= 256.
-// TMEM (M = 64 layout: row m lives in lane (m % 16) + 32 * (m / 16) of a half):
+// K/V tiles stream through an NST-stage ring; a stage is released once P.V of its tile is done.
+// TMEM (M = 64 layout: row m lives in lane (m % 16) + 32 * (m / 16) of a lane half):
 //   lane half 0 (lanes 0-15 of each quadrant): O, columns [0, dv)
-//   lane half 1 (lanes 16-31 of each quadrant): S double buffer, columns [0, 64) and [64, 128)
+//   lane half 1 (lanes 16-31 of each quadrant): S double buffer, columns [0, BK) and [BK, 2 BK)
 // Warps: 0-1 softmax (lanes 16-31 hold S rows, lanes 0-15 the matching O rows), 2 TMA producer,
 // 3 TMEM allocator + MMA issuer.
-template <int DCH, int NPIECE>
+template <int DCH, int NPIECE, int BK, int NST>
 struct DecodeTnCfg {
-  static constexpr int BK = 64;                  // keys per tile (MMA N of S)
-  static constexpr int KCH = BK * 128;           // one 64-key x 128-byte chunk
+  static constexpr int KCH = BK * 128;           // one BK-key x 128-byte chunk
   static constexpr int STAGE = DCH * KCH;
   static constexpr int QCH = 32 * 128;           // 32 query rows x 128 bytes
-  static constexpr int PB = 32 * 128;            // P tile: 32 rows x 64 keys bf16
+  static constexpr int PB = 32 * 128;            // P tile: 32 rows x (<= 64) keys bf16, 128-B rows
   static constexpr int OFF_KV = 0;
-  static constexpr int OFF_Q = OFF_KV + 2 * STAGE;
+  static constexpr int OFF_Q = OFF_KV + NST * STAGE;
   static constexpr int OFF_P = OFF_Q + DCH * QCH;   // right after Q: rows 32..63 of the M=64 reads
   static constexpr int OFF_PAD = OFF_P + 2 * PB;    // 4 KB of slack read as rows 32..63 of P1
   static constexpr int OFF_BAR = OFF_PAD + 4096;
-  // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int N_BARS = 12;
+  // barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int N_BARS = 1 + 2 * NST + 7;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t S_LANE = 16;
   static constexpr int THREADS = 128;
+  static_assert(BK == 32 || BK == 48 || BK == 64, "key tile");
+  static_assert(OFF_Q % 1024 == 0 && KCH % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int DCH, int NPIECE>
-__global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
+// Load BK (32, 48 or 64) fp32 columns of the calling warp's lanes from TMEM.
+template <int BK>
+__device__ __forceinline__ void tmem_ld_keys(uint32_t taddr, float (&x)[64]) {
+  float a[32];
+  tmem_ld32(taddr, a);
+#pragma unroll
+  for (int e = 0; e < 32; ++e) x[e] = a[e];
+  if constexpr (BK == 64) {
+    float b[32];
+    tmem_ld32(taddr + 32, b);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[32 + e] = b[e];
+  } else if constexpr (BK == 48) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr + 32));
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[32 + e] = __uint_as_float(r[e]);
+  }
+}
+
+template <int DCH, int NPIECE, int BK, int NST>
+__global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
     decode_tn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                      const DecodeParams p) {
-  using C = DecodeTnCfg<DCH, NPIECE>;
+  using C = DecodeTnCfg<DCH, NPIECE, BK, NST>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -606,15 +634,15 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
   const long long row0 = ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
   const int j_begin = split * p.chunk;
   const int j_end = min(p.Lk, j_begin + p.chunk);
-  const int n_tiles = j_end > j_begin ? (j_end - j_begin + C::BK - 1) / C::BK : 0;
+  const int n_tiles = j_end > j_begin ? (j_end - j_begin + BK - 1) / BK : 0;
   const int off = p.Lk - p.Lq;
   const int NW = p.dv / NPIECE;  // columns per O piece (multiple of 64)
   const uint32_t TMEM_COLS = p.dv <= 128 ? 128u : (p.dv <= 256 ? 256u : 512u);
 
   const uint32_t bar_q = base + C::OFF_BAR;
   const uint32_t bar_kv_full = bar_q + 8;
-  const uint32_t bar_kv_empty = bar_kv_full + 16;
-  const uint32_t bar_s_full = bar_kv_empty + 16;
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * NST;
+  const uint32_t bar_s_full = bar_kv_empty + 8 * NST;
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_pv_done = bar_p_full + 16;
   const uint32_t bar_drain = bar_pv_done + 16;
@@ -622,9 +650,11 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(bar_kv_full + 8 * i, 1);
       mbar_init(bar_kv_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar_s_full + 8 * i, 1);
       mbar_init(bar_p_full + 8 * i, 64);
       mbar_init(bar_pv_done + 8 * i, 1);
@@ -653,25 +683,25 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
       int t = 0;
       bool ok = true;
       for (; t < n_tiles; ++t) {
-        const int s = t & 1;
-        if (t >= 2) ok = mbar_wait(bar_kv_empty + 8 * s, ((t >> 1) & 1) ^ 1, 41);
+        const int s = t % NST;
+        if (t >= NST) ok = mbar_wait(bar_kv_empty + 8 * s, ((t / NST) & 1) ^ 1, 41);
         if (!ok) break;
         const uint32_t full = bar_kv_full + 8 * s;
         mbar_arrive_expect_tx(full, C::STAGE);
 #pragma unroll
         for (int c = 0; c < DCH; ++c)
-          tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * C::BK, z);
+          tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * BK, z);
       }
       if (!ok) {
         mbar_wait_drain(bar_q, 0);
-        for (int u = max(0, t - 2); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u & 1), (u >> 1) & 1);
+        for (int u = max(0, t - NST); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u % NST), (u / NST) & 1);
       }
     }
   } else if (warp == 3) {
     // ------------------------------- MMA issuer -------------------------------
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(64, C::BK, false, false);  // S = Q.K^T
-      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);         // O += P.V
+      constexpr uint32_t idesc_s = make_idesc_bf16(64, BK, false, false);  // S = Q.K^T
+      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);      // O += P.V
       const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL;
       bool ok = mbar_wait(bar_q, 0, 42);
       bool issued = false;
@@ -679,10 +709,10 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
         ok = mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 43);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (tt & 1) * C::STAGE;
+        const uint32_t kb = base + C::OFF_KV + (tt % NST) * C::STAGE;
         const uint32_t pb = base + C::OFF_P + (tt & 1) * C::PB;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk) {
+        for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
 #pragma unroll
           for (int h = 0; h < NPIECE; ++h) {
@@ -691,19 +721,19 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
             mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(bar_kv_empty + 8 * (tt & 1));
+        mma_commit(bar_kv_empty + 8 * (tt % NST));
         mma_commit(bar_pv_done + 8 * (tt & 1));
       };
       for (int t = 0; t < n_tiles && ok; ++t) {
-        ok = mbar_wait(bar_kv_full + 8 * (t & 1), (t >> 1) & 1, 44);
+        ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (t & 1) * C::STAGE;
+        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE;
 #pragma unroll
         for (int kk = 0; kk < 4 * DCH; ++kk) {
           const uint64_t ad = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
           const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          mma_ss(s_tmem + (t & 1) * C::BK, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(s_tmem + (t & 1) * BK, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         issued = true;
         mma_commit(bar_s_full + 8 * (t & 1));
@@ -730,22 +760,19 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      float x[2][32];
-      tmem_ld32(tw + C::S_COL + (t & 1) * C::BK, x[0]);
-      tmem_ld32(tw + C::S_COL + (t & 1) * C::BK + 32, x[1]);
+      float x[64];
+      tmem_ld_keys<BK>(tw + C::S_COL + (t & 1) * BK, x);
       tmem_wait_ld();
-      const int k0 = j_begin + t * C::BK;
+      const int k0 = j_begin + t * BK;
       int lim = j_end - 1;
       if (p.causal) lim = min(lim, qi + off);
       const int rem = lim - k0;  // keys c <= rem of this tile are visible
       float mx = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (32 * h + e > rem) x[h][e] = -INFINITY;
-          mx = fmaxf(mx, x[h][e]);
-        }
+      for (int e = 0; e < BK; ++e) {
+        if (e > rem) x[e] = -INFINITY;
+        mx = fmaxf(mx, x[e]);
+      }
       const float m_tile = mx * c2;
       float alpha = 1.f;
       if (m_tile != -INFINITY) {
@@ -766,14 +793,12 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE>::THREADS, 1)
       float sum = 0.f;
       uint8_t* prow = smem + C::OFF_P + (t & 1) * C::PB;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // 8 keys per 16-byte unit
+      for (int u = 0; u < BK / 8; ++u) {  // 8 keys per 16-byte unit
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float v0 = x[u >> 2][(8 * u + 2 * e) & 31];
-          const float v1 = x[u >> 2][(8 * u + 2 * e + 1) & 31];
-          const float p0 = ex2_approx(fmaf(v0, c2, -m_ref));
-          const float p1 = ex2_approx(fmaf(v1, c2, -m_ref));
+          const float p0 = ex2_approx(fmaf(x[8 * u + 2 * e], c2, -m_ref));
+          const float p1 = ex2_approx(fmaf(x[8 * u + 2 * e + 1], c2, -m_ref));
           sum += p0 + p1;
           w4[e] = pack_bf16x2(p0, p1);
         }

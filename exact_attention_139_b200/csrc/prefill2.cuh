@@ -1,0 +1,388 @@
+// prefill2.cuh -- persistent forward (prefill) attention on sm_100a with two query tiles per CTA.
+//
+// Same arithmetic as prefill.cuh (S = Q.K^T, running-max / running-sum softmax, O += P.V with
+// fp32 accumulators in TMEM; the standard flow of the FlashMLA-ETAP summary, "Mecanismo Central",
+// item 1, evaluated tile by tile on chip as in "Activar Flash Attention con llama.cpp", "Que es
+// Flash Attention"), organised so the tensor core never waits for the exponentials:
+//
+//   * a work unit is a pair of 128-row query tiles (A = rows q0.., B = rows q0+128..) of one
+//     (batch, head); both share every K/V tile;
+//   * two softmax warpgroups (A: warps 0-3, B: warps 4-7) each own one tile, one query row per
+//     thread (TMEM lane); while one computes exponentials the MMA warp runs the other's products:
+//         S_A(0) S_B(0) | PV_A(0) S_A(1) | PV_B(0) S_B(1) | PV_A(1) S_A(2) | ...
+//   * P (bf16) is written back into TMEM over the S columns it came from, and P.V takes its A
+//     operand from TMEM; shared memory holds only Q_A, Q_B and a deep K/V ring;
+//   * the grid is persistent (one CTA per SM), units are handed out round-robin in heaviest-first
+//     order (causal: last query tiles first), and every barrier phase carries across units.
+// Warps: 0-7 softmax, 8 TMA producer, 9 TMEM allocator + MMA issuer.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+struct Prefill2Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int B, Hq, Hkv, Lq, Lk, G;
+  int n_pairs;  // ceil(ceil(Lq / 128) / 2)
+  int n_units;  // n_pairs * B * Hq
+  int causal;
+  float scale_log2;
+};
+
+template <int D>
+struct Prefill2Cfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int DC = D / 64;
+  static constexpr int CHUNK = 128 * 128;
+  static constexpr int Q_BYTES = DC * CHUNK;
+  static constexpr int KV_BYTES = DC * CHUNK;
+  static constexpr int NS = (D == 128) ? 4 : 6;
+  static constexpr int OFF_Q = 0;  // Q_A, then Q_B
+  static constexpr int OFF_KV = 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+  // q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], o_free[2], drain
+  static constexpr int N_BARS = 2 + 2 * NS + 8 + 1;
+  static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  __host__ __device__ static constexpr uint32_t s_col(int x) { return (uint32_t)(128 * x); }
+  __host__ __device__ static constexpr uint32_t o_col(int x) { return (uint32_t)(256 + D * x); }
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Number of 128-key tiles query tile [qr0, qr0 + 128) needs (0 when the tile is past Lq).
+__device__ __forceinline__ int prefill_kv_tiles(const Prefill2Params& p, int qr0) {
+  if (qr0 >= p.Lq) return 0;
+  int n = (p.Lk + 127) / 128;
+  if (p.causal) {
+    const int last = min(qr0 + 127, p.Lq - 1);
+    n = min(n, (last + (p.Lk - p.Lq)) / 128 + 1);
+  }
+  return n;
+}
+
+struct UnitCoords {
+  int b, h, q0;
+};
+
+__device__ __forceinline__ UnitCoords prefill_unit(const Prefill2Params& p, int u) {
+  const int BH = p.B * p.Hq;
+  const int i = u / BH, bh = u % BH;
+  UnitCoords c;
+  c.b = bh / p.Hq;
+  c.h = bh % p.Hq;
+  c.q0 = (p.n_pairs - 1 - i) * 256;  // heaviest (last) pairs first
+  return c;
+}
+
+template <int D>
+__global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
+    prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const Prefill2Params p) {
+  using C = Prefill2Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const uint32_t bar_q_full = base + C::OFF_BAR;
+  const uint32_t bar_q_empty = bar_q_full + 8;
+  const uint32_t bar_kv_full = bar_q_empty + 8;
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * C::NS;
+  const uint32_t bar_s_full = bar_kv_empty + 8 * C::NS;  // [2]
+  const uint32_t bar_p_full = bar_s_full + 16;           // [2]
+  const uint32_t bar_o_ready = bar_p_full + 16;          // [2]
+  const uint32_t bar_o_free = bar_o_ready + 16;          // [2]
+  const uint32_t bar_drain = bar_o_free + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar_kv_full + 8 * s, 1);
+      mbar_init(bar_kv_empty + 8 * s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_s_full + 8 * x, 1);
+      mbar_init(bar_p_full + 8 * x, 128);
+      mbar_init(bar_o_ready + 8 * x, 1);
+      mbar_init(bar_o_free + 8 * x, 128);
+    }
+    mbar_init(bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 8) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      bool ok = true;
+      int kv_t = 0, qc = 0;
+      auto load_kv = [&](const CUtensorMap* m, int tile, int zkv) {
+        const int s = kv_t % C::NS;
+        if (kv_t >= C::NS) ok = mbar_wait(bar_kv_empty + 8 * s, ((kv_t / C::NS) & 1) ^ 1, 61);
+        if (!ok) return;
+        const uint32_t full = bar_kv_full + 8 * s;
+        mbar_arrive_expect_tx(full, C::KV_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DC; ++c)
+          tma_load_3d(base + C::OFF_KV + s * C::KV_BYTES + c * C::CHUNK, m, full, 64 * c, tile * C::BN, zkv);
+        ++kv_t;
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const UnitCoords uc = prefill_unit(p, u);
+        const int nA = prefill_kv_tiles(p, uc.q0), nB = prefill_kv_tiles(p, uc.q0 + 128);
+        const int n = max(nA, nB);
+        if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
+        if (!ok) break;
+        const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
+        mbar_arrive_expect_tx(bar_q_full, (nB > 0 ? 2 : 1) * C::Q_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
+        if (nB > 0) {
+#pragma unroll
+          for (int c = 0; c < C::DC; ++c)
+            tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+        }
+        ++qc;
+        for (int j = 0; j < n && ok; ++j) {
+          load_kv(&tm_k, j, zkv);
+          if (ok) load_kv(&tm_v, j, zkv);
+        }
+      }
+      if (!ok) {
+        if (qc > 0) mbar_wait_drain(bar_q_full, (qc - 1) & 1);
+        for (int u = max(0, kv_t - C::NS); u < kv_t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u % C::NS), (u / C::NS) & 1);
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(C::BM, C::BN, false, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(C::BM, D, false, true);
+      bool ok = true, issued = false;
+      int kv_t = 0, qc = 0;
+      int p_cnt[2] = {0, 0}, units_done[2] = {0, 0};
+      auto wait_stage = [&](int idx, uint32_t site) {
+        ok = mbar_wait(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site);
+        if (ok) tc_fence_after();
+      };
+      auto issue_s = [&](int x, int kidx) {
+        const uint32_t kb = base + C::OFF_KV + (kidx % C::NS) * C::KV_BYTES;
+        const uint32_t qb = base + C::OFF_Q + x * C::Q_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = make_sdesc(qb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+          mma_ss(tmem + C::s_col(x), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s_full + 8 * x);
+        issued = true;
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const UnitCoords uc = prefill_unit(p, u);
+        int nX[2];
+        nX[0] = prefill_kv_tiles(p, uc.q0);
+        nX[1] = prefill_kv_tiles(p, uc.q0 + 128);
+        const int n = max(nX[0], nX[1]);
+        ok = mbar_wait(bar_q_full, qc & 1, 63);
+        if (!ok) break;
+        ++qc;
+        tc_fence_after();
+        wait_stage(kv_t, 64);  // K_0
+        if (!ok) break;
+        for (int x = 0; x < 2; ++x)
+          if (nX[x] > 0) issue_s(x, kv_t);
+        mma_commit(bar_kv_empty + 8 * (kv_t % C::NS));
+        if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
+        for (int j = 0; j < n && ok; ++j) {
+          const int vi = kv_t + 2 * j + 1, ki = kv_t + 2 * j + 2;
+          wait_stage(vi, 65);  // V_j
+          if (!ok) break;
+          bool k_next = false;
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j >= nX[x]) continue;
+            if (j == 0 && units_done[x] > 0) {
+              ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
+              if (!ok) break;
+            }
+            ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
+            if (!ok) break;
+            ++p_cnt[x];
+            tc_fence_after();
+            const uint32_t vb = base + C::OFF_KV + (vi % C::NS) * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::BN / 16; ++kk) {
+              const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
+              // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
+              mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            if (j + 1 < nX[x]) {
+              if (!k_next) {
+                wait_stage(ki, 68);  // K_{j+1}
+                if (!ok) break;
+                k_next = true;
+              }
+              issue_s(x, ki);
+            }
+            if (j == nX[x] - 1) {
+              mma_commit(bar_o_ready + 8 * x);
+              ++units_done[x];
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar_kv_empty + 8 * (vi % C::NS));
+          if (k_next) mma_commit(bar_kv_empty + 8 * (ki % C::NS));
+          // Q may be reloaded once the last S of this unit (issued in iteration n-2) is done
+          if (j == n - 2) mma_commit(bar_q_empty);
+        }
+        if (!ok) break;
+        kv_t += 2 * n;
+      }
+      if (!ok && issued) {
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+    }
+  } else {
+    // --------------------------- softmax warpgroups (warps 0-3: A, 4-7: B) ---------------------------
+    const int x = warp >> 2;
+    const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
+    const uint32_t tw = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_col = C::s_col(x), o_col = C::o_col(x);
+    const float c2 = p.scale_log2;
+    const int off = p.Lk - p.Lq;
+    int s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const UnitCoords uc = prefill_unit(p, u);
+      const int qx0 = uc.q0 + 128 * x;
+      const int nt = prefill_kv_tiles(p, qx0);
+      if (nt == 0) continue;
+      const int row = qx0 + r;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        ok = mbar_wait(bar_s_full + 8 * x, s_cnt & 1, 69);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float s[4][32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tw + s_col + 32 * c4, s[c4]);
+        tmem_wait_ld();
+        const int kv0 = j * C::BN;
+        if (kv0 + C::BN > p.Lk || (p.causal && kv0 + C::BN - 1 > qx0 + off)) {
+          int lim = p.Lk - 1;
+          if (p.causal) lim = min(lim, row + off);
+          const int rem = lim - kv0;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (32 * c4 + e > rem) s[c4][e] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, s[c4][e]);
+        const float m_tile = mx * c2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_used = m_tile;
+        } else if (m_tile > m_used + kRescaleLog2) {
+          alpha = ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+          rescale = true;
+        }
+        const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
+        l *= alpha;
+        float sum = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float v0 = s[2 * half + (e >> 4)][(2 * e) & 31];
+            const float v1 = s[2 * half + (e >> 4)][(2 * e + 1) & 31];
+            const float p0 = ex2_approx(fmaf(v0, c2, -m_ref));
+            const float p1 = ex2_approx(fmaf(v1, c2, -m_ref));
+            sum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // P overwrites the S columns it came from: keys 64*half .. 64*half + 63
+          tmem_st32u(tw + s_col + 32 * half, pk);
+        }
+        l += sum;
+        // s_full of tile j also covers P.V of tile j-1, so O is stable here
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            float o[32];
+            tmem_ld32(tw + o_col + 32 * c4, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tw + o_col + 32 * c4, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p_full + 8 * x);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16, LSE
+      ok = mbar_wait(bar_o_ready + 8 * x, o_cnt & 1, 70);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++o_cnt;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool in_range = row < p.Lq;
+      __nv_bfloat16* orow = p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + (in_range ? row : 0)) * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        float o[32];
+        tmem_ld32(tw + o_col + 32 * c4, o);
+        tmem_wait_ld();
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l),
+                                pack_bf16x2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l),
+                                pack_bf16x2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l),
+                                pack_bf16x2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
+        }
+      }
+      if (in_range && p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = (m_used + log2f(l)) * kLn2;
+      tc_fence_before();
+      mbar_arrive(bar_o_free + 8 * x);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn
