@@ -565,11 +565,16 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
 // K/V tiles stream through an NST-stage ring; a stage is released once P.V of its tile is done.
 // TMEM (M = 64 layout: row m lives in lane (m % 16) + 32 * (m / 16) of a lane half):
 //   lane half 0 (lanes 0-15 of each quadrant): O, columns [0, dv)
-//   lane half 1 (lanes 16-31 of each quadrant): S double buffer, columns [0, BK) and [BK, 2 BK)
+//   lane half 1 (lanes 16-31 of each quadrant): S double buffer of NACC partial tiles,
+//                columns [(b * NACC + a) * BK, ... + BK) for buffer b, partial a
 // Warps: 0-1 softmax (lanes 16-31 hold S rows, lanes 0-15 the matching O rows), 2 TMA producer,
-// 3 TMEM allocator + MMA issuer.
+// 3 TMEM allocator + P.V issuer, 4 .. 3 + NACC S issuers.
 template <int DCH, int NPIECE, int BK, int NST>
 struct DecodeTnCfg {
+  // S = Q.K^T is accumulated in NACC independent TMEM tiles (chunk c of the d columns goes to
+  // tile c % NACC) issued interleaved: back-to-back MMAs into one accumulator serialise on its
+  // latency, independent ones overlap. The softmax adds the partial tiles.
+  static constexpr int NACC = (DCH % 3 == 0) ? 3 : ((DCH % 2 == 0) ? 2 : 1);
   static constexpr int KCH = BK * 128;           // one BK-key x 128-byte chunk
   static constexpr int STAGE = DCH * KCH;
   static constexpr int QCH = 32 * 128;           // 32 query rows x 128 bytes
@@ -579,14 +584,19 @@ struct DecodeTnCfg {
   static constexpr int OFF_P = OFF_Q + DCH * QCH;   // right after Q: rows 32..63 of the M=64 reads
   static constexpr int OFF_PAD = OFF_P + 2 * PB;    // 4 KB of slack read as rows 32..63 of P1
   static constexpr int OFF_BAR = OFF_PAD + 4096;
-  // barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int N_BARS = 1 + 2 * NST + 7;
+  // barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], pv_done[2],
+  // drain[1 + NACC] (one per MMA-issuing warp)
+  static constexpr int N_BARS = 1 + 2 * NST + 6 + 1 + NACC;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
   static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t S_LANE = 16;
-  static constexpr int THREADS = 128;
+  // warps: 0-1 softmax, 2 TMA producer, 3 TMEM allocator + P.V issuer, 4.. S issuers (one per
+  // partial accumulator): one thread issuing tcgen05.mma back to back is limited by its own
+  // instruction latency for these small shapes, so the S products are spread over NACC warps.
+  static constexpr int THREADS = 32 * (4 + NACC);
   static_assert(BK == 32 || BK == 48 || BK == 64, "key tile");
+  static_assert(2 * NACC * BK <= 512, "S partial tiles fit in one lane half");
   static_assert(OFF_Q % 1024 == 0 && KCH % 1024 == 0, "128-byte swizzle atoms need 1 KB alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -655,11 +665,11 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
       mbar_init(bar_kv_empty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_s_full + 8 * i, 1);
+      mbar_init(bar_s_full + 8 * i, C::NACC);  // one commit per S issuer
       mbar_init(bar_p_full + 8 * i, 64);
       mbar_init(bar_pv_done + 8 * i, 1);
     }
-    mbar_init(bar_drain, 1);
+    for (int i = 0; i <= C::NACC; ++i) mbar_init(bar_drain + 8 * i, 1);
     fence_mbar_init();
   }
   if (warp == 3) {
@@ -697,20 +707,52 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
         for (int u = max(0, t - NST); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u % NST), (u / NST) & 1);
       }
     }
-  } else if (warp == 3) {
-    // ------------------------------- MMA issuer -------------------------------
+  } else if (warp >= 4) {
+    // -------------------- S issuers: partial a = chunks a, a + NACC, ... --------------------
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_s = make_idesc_bf16(64, BK, false, false);  // S = Q.K^T
-      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);      // O += P.V
-      const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL;
+      const int a = warp - 4;
+      const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL + a * BK;
+      const uint64_t qdesc = make_sdesc(base + C::OFF_Q + a * C::QCH, 16, 1024, kSwizzle128B);
       bool ok = mbar_wait(bar_q, 0, 42);
       bool issued = false;
-      auto pv = [&](int tt) {
-        ok = mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 43);
-        if (!ok) return;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
+        // S buffer (t & 1) was last read by the softmax of tile t - 2
+        if (ok && t >= 2) ok = mbar_wait(bar_p_full + 8 * (t & 1), ((t - 2) >> 1) & 1, 50);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (tt % NST) * C::STAGE;
-        const uint32_t pb = base + C::OFF_P + (tt & 1) * C::PB;
+        const uint64_t kdesc = make_sdesc(base + C::OFF_KV + (t % NST) * C::STAGE + a * C::KCH, 16, 1024, kSwizzle128B);
+        const uint32_t d = s_tmem + (t & 1) * C::NACC * BK;
+#pragma unroll
+        for (int i = 0; i < DCH / C::NACC; ++i) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            // descriptor start addresses advance by whole 16-byte units
+            const uint64_t qa = qdesc + (uint64_t)((i * C::NACC * C::QCH + ks * 32) >> 4);
+            const uint64_t kb = kdesc + (uint64_t)((i * C::NACC * C::KCH + ks * 32) >> 4);
+            mma_ss(d, qa, kb, idesc_s, (i > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        issued = true;
+        mma_commit(bar_s_full + 8 * (t & 1));
+      }
+      if (!ok && issued) {
+        mma_commit(bar_drain + 8 * (1 + a));
+        mbar_wait_drain(bar_drain + 8 * (1 + a), 0);
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------- P.V issuer -------------------------------
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);  // O += P.V
+      bool ok = true, issued = false;
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE;
+        const uint32_t pb = base + C::OFF_P + (t & 1) * C::PB;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
@@ -718,28 +760,15 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
           for (int h = 0; h < NPIECE; ++h) {
             // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
             const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
-            mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tmem + h * NW, ad, bd, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(bar_kv_empty + 8 * (tt % NST));
-        mma_commit(bar_pv_done + 8 * (tt & 1));
-      };
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < 4 * DCH; ++kk) {
-          const uint64_t ad = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          mma_ss(s_tmem + (t & 1) * BK, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-        }
         issued = true;
-        mma_commit(bar_s_full + 8 * (t & 1));
-        if (t > 0) pv(t - 1);
+        // the S products of this tile completed before its softmax started, so this commit
+        // also covers every read of the stage
+        mma_commit(bar_kv_empty + 8 * (t % NST));
+        mma_commit(bar_pv_done + 8 * (t & 1));
       }
-      if (ok) pv(n_tiles - 1);
       if (!ok && issued) {
         mma_commit(bar_drain);
         mbar_wait_drain(bar_drain, 0);
@@ -761,7 +790,15 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       float x[64];
-      tmem_ld_keys<BK>(tw + C::S_COL + (t & 1) * BK, x);
+      tmem_ld_keys<BK>(tw + C::S_COL + (t & 1) * C::NACC * BK, x);
+#pragma unroll
+      for (int a = 1; a < C::NACC; ++a) {
+        float y[64];
+        tmem_ld_keys<BK>(tw + C::S_COL + ((t & 1) * C::NACC + a) * BK, y);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < BK; ++e) x[e] += y[e];
+      }
       tmem_wait_ld();
       const int k0 = j_begin + t * BK;
       int lim = j_end - 1;

@@ -297,11 +297,16 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             for (int e = 0; e < 32; ++e)
               if (32 * c4 + e > rem) s[c4][e] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max: two independent chains of three-input maxima
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, s[c4][e]);
+          for (int e = 0; e < 32; e += 4) {
+            mx0 = fmax3(mx0, s[c4][e], s[c4][e + 1]);
+            mx1 = fmax3(mx1, s[c4][e + 2], s[c4][e + 3]);
+          }
+        const float mx = fmaxf(mx0, mx1);
         const float m_tile = mx * c2;
         float alpha = 1.f;
         bool rescale = false;
@@ -314,22 +319,29 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         }
         const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
         l *= alpha;
-        float sum = 0.f;
+        // p = 2^(s * c2 - m_ref) on key pairs: packed fma, two ex2, packed sum, bf16x2 pack
+        const uint64_t c2x2 = f2_pack(c2, c2), nm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+        for (int q4 = 0; q4 < 4; ++q4) {  // 32 keys -> 16 packed columns at a time
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v0 = s[2 * half + (e >> 4)][(2 * e) & 31];
-            const float v1 = s[2 * half + (e >> 4)][(2 * e + 1) & 31];
-            const float p0 = ex2_approx(fmaf(v0, c2, -m_ref));
-            const float p1 = ex2_approx(fmaf(v1, c2, -m_ref));
-            sum += p0 + p1;
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t xv = ffma2(f2_pack(s[q4][2 * e], s[q4][2 * e + 1]), c2x2, nm2);
+            float x0, x1;
+            f2_unpack(xv, x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (e & 1) acc1 = fadd2(acc1, f2_pack(p0, p1));
+            else acc0 = fadd2(acc0, f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
-          // P overwrites the S columns it came from: keys 64*half .. 64*half + 63
-          tmem_st32u(tw + s_col + 32 * half, pk);
+          // P overwrites the S columns it came from: keys 32*q4 .. 32*q4 + 31
+          tmem_st16u(tw + s_col + 16 * q4, pk);
         }
+        float a0, a1, b0, b1;
+        f2_unpack(acc0, a0, a1);
+        f2_unpack(acc1, b0, b1);
+        const float sum = (a0 + a1) + (b0 + b1);
         l += sum;
         // s_full of tile j also covers P.V of tile j-1, so O is stable here
         if (__any_sync(0xffffffffu, rescale)) {
