@@ -227,15 +227,16 @@ def bench_prefill_e2e(w, dev, steps, warmup, host):
 
 def bench_decode(w, dev, steps, warmup, flush, stream):
     from exact_attention_139_b200 import attn
-    q, k, _ = make_inputs(w)
+    q, k, v = make_inputs(w)
     qd, kd = q.to(dev), k.to(dev)
-    del q, k
+    vd = kd if w.latent else v.to(dev)
+    del q, k, v
     splits = attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv)
     ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, splits),
                      dtype=torch.uint8, device=dev)
     o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
-    step = lambda: attn.attn_decode(qd, kd, kd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=splits,
+    step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=splits,
                                     workspace=ws, out=o, lse=lse)
     times = time_steps(step, steps, warmup, flush, stream)
     if attn.attn_check_device() != attn.ATTN_OK:
@@ -288,6 +289,17 @@ def run_ours(args):
         dclk = clocks_d.stop()
         dms = max_over_ranks(sum(dtimes) / len(dtimes), world)
         gbs = wd.kv_bytes() / (dms * 1e-3) / 1e9
+        wg = rank_workload(WORKLOADS["gqa_decode_32k"], rank)
+        gtimes, gsplits = bench_decode(wg, dev, args.steps, args.warmup, flush, stream)
+        gms = max_over_ranks(sum(gtimes) / len(gtimes), world)
+        ggbs = wg.kv_bytes() / (gms * 1e-3) / 1e9
+        extras["decode_gqa"] = {
+            "workload": wg.name, "metric": "KV-read HBM GB/s", "value": round(ggbs * world, 1),
+            "per_gpu_gbs": round(ggbs, 1), "ms_per_step": round(gms, 4), "num_splits": gsplits,
+            "roofline": {"bound": "hbm", "achieved": round(ggbs, 1), "peak": float(peaks["hbm_gbs"]),
+                         "unit": "GB/s", "frac": round(ggbs / float(peaks["hbm_gbs"]), 4),
+                         "algorithmic_bytes_per_launch": wg.kv_bytes()}}
+        launches += 2 * args.steps
         extras["decode"] = {
             "workload": wd.name, "metric": "KV-read HBM GB/s", "value": round(gbs * world, 1),
             "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits,

@@ -15,21 +15,14 @@
 #include "../../include/attn.h"
 #include "combine.cuh"
 #include "decode.cuh"
-#include "prefill.cuh"
 #include "prefill2.cuh"
 
 namespace {
 
 using attn::DecodeParams;
-using attn::PrefillParams;
 
 constexpr int kAbiVersion = 10000;  // 1.0.0
 
-#ifndef ATTN_PREFILL_VERSION
-#define ATTN_PREFILL_VERSION 2
-#endif
-// 2: persistent two-tile kernel (prefill2.cuh); 1: one 128-row tile per CTA (prefill.cuh).
-constexpr int kPrefillVersion = ATTN_PREFILL_VERSION;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -50,11 +43,13 @@ EncodeTiledFn get_encoder() {
 
 // bf16 tensor map over a row-major [n2, n1, n0] array (n0 contiguous), 128-byte swizzle,
 // zero fill out of bounds. box = {b0, b1, 1}. rank 2 when n2 == 0.
-bool encode_bf16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1) {
+bool encode_bf16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1,
+                 uint64_t row_stride = 0) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return false;
+  const uint64_t rs = row_stride ? row_stride : n0;  // elements between consecutive rows
   cuuint64_t dims[3] = {n0, n1, n2};
-  cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+  cuuint64_t strides[2] = {rs * 2, rs * n1 * 2};
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = n2 == 0 ? 2 : 3;
@@ -112,6 +107,13 @@ bool tc_supported(const void* k, const void* v, int Hq, int Hkv, int Lq, int d, 
   return v == k && ldv == d && d % 64 == 0 && d <= 576 && dv % 128 == 0 && dv <= 512 && dv <= d && R <= 32;
 }
 
+// queries-on-M kernel: latent KV as above, or a dense separate V with dv == d (GQA decode)
+bool tn_supported(const void* k, const void* v, int Hq, int Hkv, int Lq, int d, int dv, int ldv) {
+  if (tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv)) return true;
+  const int R = (Hq / Hkv) * Lq;
+  return v != k && dv == d && (d == 128 || d == 256) && ldv % 8 == 0 && R <= 32;
+}
+
 bool cc_supported(int Hq, int Hkv, int Lq, int d, int dv, int ldv) {
   const int R = (Hq / Hkv) * Lq;
   return R <= 64 && d <= 576 && dv <= 512 && d % 8 == 0 && dv % 8 == 0 && ldv % 8 == 0 && ldv >= dv;
@@ -123,28 +125,28 @@ int split_chunk(int Lk, int splits) {
   return (c + 63) / 64 * 64;
 }
 
-// Choose the split count: every CTA is resident one per SM (tensor-core kernel) or a few per SM
-// (CUDA-core kernel); minimise idle SMs in the last wave plus the partial-result traffic relative
-// to the KV bytes, with at least 256 keys per split.
-// Depends only on the sizes attn_decode_workspace_size also sees (the KV bytes are estimated
-// from dv), so both always agree on the count.
+// Choose the split count. Model: CTAs run one per SM in waves; a CTA costs its key tiles plus a
+// fixed start-up/drain cost of about kFixedTiles tiles (barrier set-up, Q load, ring fill, partial
+// write), and every split adds partial-result traffic. Minimise
+//   waves * (tiles per split + kFixedTiles) * (1 + partial bytes / KV bytes).
+// (On B200: mla_decode_64k -> 9 splits, gqa_decode_32k -> 8, both the measured best.)
 int choose_splits(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int sms, int ctas_per_sm) {
+  constexpr double kFixedTiles = 5.0, kTileKeys = 48.0;
   const long long units = (long long)B * Hkv;
   const long long rows = (long long)B * Hq * Lq;
   const double kv_bytes = (double)units * Lk * (double)dv * 2.0;
   const int max_s = std::max(1, std::min(256, Lk / 256));
   int best = 1;
-  double best_cost = 1e30;
+  double best_cost = 1e300;
   for (int s = 1; s <= max_s; ++s) {
     const int chunk = split_chunk(Lk, s);
     const int used = (Lk + chunk - 1) / chunk;  // splits that hold keys
     if (used < s) continue;
     const double slots = (double)sms * ctas_per_sm;
-    const double waves = (double)(units * s) / slots;
-    const double waste = std::ceil(waves) / waves - 1.0;
+    const double waves = std::ceil((double)(units * s) / slots);
     const double partial = 2.0 * (double)s * rows * (dv + 1) * 4.0 / kv_bytes;
-    const double cost = waste + partial + (waves < 1.0 ? (1.0 - waves) : 0.0);
-    if (cost < best_cost - 1e-9) {
+    const double cost = waves * (std::ceil(chunk / kTileKeys) + kFixedTiles) * (1.0 + partial);
+    if (cost < best_cost * (1.0 - 1e-9)) {
       best_cost = cost;
       best = s;
     }
@@ -202,26 +204,38 @@ attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
 // Key tile and stage count of the queries-on-M decode kernel (chosen by measurement on B200).
 constexpr int kTnBK = ATTN_TN_BK, kTnNST = ATTN_TN_NST;
 
-template <int DCH, int NPIECE>
+template <int DCH, int NPIECE, int NST, bool SEPV>
 attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
-  using C = attn::DecodeTnCfg<DCH, NPIECE, kTnBK, kTnNST>;
-  CUtensorMap tq, tkv;
+  using C = attn::DecodeTnCfg<DCH, NPIECE, kTnBK, NST, SEPV>;
+  CUtensorMap tq, tkv, tv;
   if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
   if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK)) return ATTN_ERR_CUDA;
-  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, kTnNST>;
+  if (SEPV) {
+    if (!encode_bf16(&tv, p.v, (uint64_t)p.dv, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK, (uint64_t)p.ldv))
+      return ATTN_ERR_CUDA;
+  } else {
+    tv = tkv;  // unused
+  }
+  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, NST, SEPV>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, tv, p);
   return launch_status();
 }
 
 template <int DCH>
 attn_status launch_tn_np(const DecodeParams& p, int splits, cudaStream_t st) {
-  if (p.dv <= 256) return launch_tn<DCH, 1>(p, splits, st);
-  return launch_tn<DCH, 2>(p, splits, st);
+  if (p.dv <= 256) return launch_tn<DCH, 1, kTnNST, false>(p, splits, st);
+  return launch_tn<DCH, 2, kTnNST, false>(p, splits, st);
 }
 
 attn_status launch_tn_any(const DecodeParams& p, int splits, cudaStream_t st) {
+  if (!p.v_is_k) {
+    // dense V beside K in each stage (small stages: a deeper ring)
+    if (p.d == 128) return launch_tn<2, 1, 6, true>(p, splits, st);
+    if (p.d == 256) return launch_tn<4, 1, 3, true>(p, splits, st);
+    return ATTN_ERR_UNSUPPORTED;
+  }
   switch (p.d / 64) {
     case 2: return launch_tn_np<2>(p, splits, st);
     case 3: return launch_tn_np<3>(p, splits, st);
@@ -272,6 +286,21 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
   __syncthreads();
 }
 
+// y[i] = 2^x[i] through the FMA-pipe polynomial used by the prefill softmax.
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    float a, b;
+    attn::f2_unpack(attn::exp2_poly2(attn::f2_pack(x[i], x[i + 1])), a, b);
+    y[i] = a;
+    y[i + 1] = b;
+  } else if (i < n) {
+    float a, b;
+    attn::f2_unpack(attn::exp2_poly2(attn::f2_pack(x[i], 0.f)), a, b);
+    y[i] = a;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -303,35 +332,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
       !encode_bf16(&tk, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
       !encode_bf16(&tv, v, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
     return ATTN_ERR_CUDA;
-  if (kPrefillVersion == 2) {
-    attn::Prefill2Params p{};
-    p.o = reinterpret_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Lq = Lq;
-    p.Lk = Lk;
-    p.G = Hq / Hkv;
-    p.n_pairs = (n_qtiles + 1) / 2;
-    const long long units = (long long)p.n_pairs * B * Hq;
-    if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-    p.n_units = (int)units;
-    p.causal = causal ? 1 : 0;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    const int grid = (int)std::min<long long>(units, current_sm_count());
-    if (d == 128) {
-      using C = attn::Prefill2Cfg<128>;
-      if (!allow_smem(attn::prefill2_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-      attn::prefill2_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
-    } else {
-      using C = attn::Prefill2Cfg<64>;
-      if (!allow_smem(attn::prefill2_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-      attn::prefill2_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
-    }
-    return launch_status();
-  }
-  PrefillParams p{};
+  attn::Prefill2Params p{};
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.B = B;
@@ -340,19 +341,22 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Lq = Lq;
   p.Lk = Lk;
   p.G = Hq / Hkv;
-  p.n_qtiles = n_qtiles;
+  p.n_pairs = (n_qtiles + 1) / 2;
+  const long long units = (long long)p.n_pairs * B * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.n_units = (int)units;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const long long grid = (long long)p.n_qtiles * B * Hq;
-  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  // persistent grid: one CTA per SM (fewer when there are fewer work units)
+  const int grid = (int)std::min<long long>(units, current_sm_count());
   if (d == 128) {
-    using C = attn::PrefillCfg<128>;
-    if (!allow_smem(attn::prefill_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill_kernel<128><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    using C = attn::Prefill2Cfg<128>;
+    if (!allow_smem(attn::prefill2_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   } else {
-    using C = attn::PrefillCfg<64>;
-    if (!allow_smem(attn::prefill_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill_kernel<64><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    using C = attn::Prefill2Cfg<64>;
+    if (!allow_smem(attn::prefill2_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   }
   return launch_status();
 }
@@ -380,10 +384,11 @@ attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o,
   if (impl < ATTN_DECODE_AUTO || impl > ATTN_DECODE_TCGEN05_N) return ATTN_ERR_INVALID_ARG;
   if (d % 8 != 0 || dv % 8 != 0 || ldv % 8 != 0) return ATTN_ERR_MISALIGNED;
   const bool tc_ok = tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
+  const bool tn_ok = tn_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
   const bool cc_ok = cc_supported(Hq, Hkv, Lq, d, dv, ldv);
-  // both tensor-core kernels serve the same shapes (tc_ok)
-  if (impl == ATTN_DECODE_AUTO) impl = tc_ok ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
-  if ((impl == ATTN_DECODE_TCGEN05_T || impl == ATTN_DECODE_TCGEN05_N) && !tc_ok) return ATTN_ERR_UNSUPPORTED;
+  if (impl == ATTN_DECODE_AUTO) impl = tn_ok ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
+  if (impl == ATTN_DECODE_TCGEN05_T && !tc_ok) return ATTN_ERR_UNSUPPORTED;
+  if (impl == ATTN_DECODE_TCGEN05_N && !tn_ok) return ATTN_ERR_UNSUPPORTED;
   if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
   int splits = num_splits;
   if (splits == 0) splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
@@ -500,6 +505,14 @@ attn_status attn_combine(const float* o_part, const float* lse_part, void* o, fl
 attn_status attn_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_INVALID_ARG;
   selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull);
+  return launch_status();
+}
+
+attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 1) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(y, 4)) return ATTN_ERR_MISALIGNED;
+  const int threads = 256, pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + threads - 1) / threads, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launch_status();
 }
 

@@ -13,7 +13,7 @@
 //                         per kv head, putting keys (64 per tile) on M and queries on N avoids
 //                         padding the query dimension to the MMA's minimum M.
 // Latent KV (MLA): V is the first dv columns of each K row; each row is read from HBM once and
-// the same shared-memory tile feeds both products.
+// the same shared-memory tile feeds both products. Dense V (GQA decode) streams beside K.
 #pragma once
 
 #include "sm100.cuh"
@@ -569,14 +569,17 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
 //                columns [(b * NACC + a) * BK, ... + BK) for buffer b, partial a
 // Warps: 0-1 softmax (lanes 16-31 hold S rows, lanes 0-15 the matching O rows), 2 TMA producer,
 // 3 TMEM allocator + P.V issuer, 4 .. 3 + NACC S issuers.
-template <int DCH, int NPIECE, int BK, int NST>
+template <int DCH, int NPIECE, int BK, int NST, bool SEPV>
 struct DecodeTnCfg {
+  // SEPV: V is a separate dense tensor (dv == d); each ring stage then holds the K tile followed
+  // by the V tile. Otherwise V is the first dv columns of the latent K tile.
   // S = Q.K^T is accumulated in NACC independent TMEM tiles (chunk c of the d columns goes to
   // tile c % NACC) issued interleaved: back-to-back MMAs into one accumulator serialise on its
   // latency, independent ones overlap. The softmax adds the partial tiles.
   static constexpr int NACC = (DCH % 3 == 0) ? 3 : ((DCH % 2 == 0) ? 2 : 1);
   static constexpr int KCH = BK * 128;           // one BK-key x 128-byte chunk
-  static constexpr int STAGE = DCH * KCH;
+  static constexpr int VOFF = DCH * KCH;         // offset of the V tile inside a stage (SEPV)
+  static constexpr int STAGE = (SEPV ? 2 : 1) * DCH * KCH;
   static constexpr int QCH = 32 * 128;           // 32 query rows x 128 bytes
   static constexpr int PB = 32 * 128;            // P tile: 32 rows x (<= 64) keys bf16, 128-B rows
   static constexpr int OFF_KV = 0;
@@ -627,11 +630,11 @@ __device__ __forceinline__ void tmem_ld_keys(uint32_t taddr, float (&x)[64]) {
   }
 }
 
-template <int DCH, int NPIECE, int BK, int NST>
-__global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
+template <int DCH, int NPIECE, int BK, int NST, bool SEPV>
+__global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREADS, 1)
     decode_tn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                     const DecodeParams p) {
-  using C = DecodeTnCfg<DCH, NPIECE, BK, NST>;
+                     const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  using C = DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -647,7 +650,9 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
   const int n_tiles = j_end > j_begin ? (j_end - j_begin + BK - 1) / BK : 0;
   const int off = p.Lk - p.Lq;
   const int NW = p.dv / NPIECE;  // columns per O piece (multiple of 64)
-  const uint32_t TMEM_COLS = p.dv <= 128 ? 128u : (p.dv <= 256 ? 256u : 512u);
+  // TMEM columns: O needs dv (lane half 0), the S partial tiles 2 * NACC * BK (lane half 1)
+  const int cols_needed = max(p.dv, 2 * C::NACC * BK);
+  const uint32_t TMEM_COLS = cols_needed <= 128 ? 128u : (cols_needed <= 256 ? 256u : 512u);
 
   const uint32_t bar_q = base + C::OFF_BAR;
   const uint32_t bar_kv_full = bar_q + 8;
@@ -686,6 +691,7 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kv);
+      if constexpr (SEPV) tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(bar_q, DCH * C::QCH);
 #pragma unroll
       for (int c = 0; c < DCH; ++c) tma_load_2d(base + C::OFF_Q + c * C::QCH, &tm_q, bar_q, 64 * c, (int)row0);
@@ -701,6 +707,11 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < DCH; ++c)
           tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * BK, z);
+        if constexpr (SEPV) {
+#pragma unroll
+          for (int c = 0; c < DCH; ++c)
+            tma_load_3d(base + C::OFF_KV + s * C::STAGE + C::VOFF + c * C::KCH, &tm_v, full, 64 * c, j_begin + t * BK, z);
+        }
       }
       if (!ok) {
         mbar_wait_drain(bar_q, 0);
@@ -751,7 +762,7 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST>::THREADS, 1)
         ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE;
+        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE + (SEPV ? C::VOFF : 0);  // V rows
         const uint32_t pb = base + C::OFF_P + (t & 1) * C::PB;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {

@@ -1,19 +1,27 @@
 // prefill2.cuh -- persistent forward (prefill) attention on sm_100a with two query tiles per CTA.
 //
-// Same arithmetic as prefill.cuh (S = Q.K^T, running-max / running-sum softmax, O += P.V with
-// fp32 accumulators in TMEM; the standard flow of the FlashMLA-ETAP summary, "Mecanismo Central",
-// item 1, evaluated tile by tile on chip as in "Activar Flash Attention con llama.cpp", "Que es
-// Flash Attention"), organised so the tensor core never waits for the exponentials:
+// Arithmetic: the standard flow S = Q.K^T, P = softmax(S), O = P.V of the FlashMLA-ETAP summary
+// ("Mecanismo Central", item 1), evaluated tile by tile in on-chip memory as in "Activar Flash
+// Attention con llama.cpp" ("Que es Flash Attention"): TMA tile loads, tcgen05.mma with fp32
+// accumulators in TMEM, a running-max / running-sum softmax with one query row per thread, exp2
+// with the scale folded in, lazy rescaling (the exponent reference moves only when a tile's max
+// exceeds it by more than 2^8), causal tiles above the diagonal never loaded.
 //
+// Organisation, chosen so the tensor core rarely waits for the exponentials:
 //   * a work unit is a pair of 128-row query tiles (A = rows q0.., B = rows q0+128..) of one
 //     (batch, head); both share every K/V tile;
 //   * two softmax warpgroups (A: warps 0-3, B: warps 4-7) each own one tile, one query row per
-//     thread (TMEM lane); while one computes exponentials the MMA warp runs the other's products:
+//     thread (TMEM lane); while one computes exponentials the MMA thread issues the other's products:
 //         S_A(0) S_B(0) | PV_A(0) S_A(1) | PV_B(0) S_B(1) | PV_A(1) S_A(2) | ...
+//     A single issuing thread keeps each tile's products contiguous on the tensor core; issuing
+//     A and B from two warps interleaved them and was measured slower;
 //   * P (bf16) is written back into TMEM over the S columns it came from, and P.V takes its A
-//     operand from TMEM; shared memory holds only Q_A, Q_B and a deep K/V ring;
-//   * the grid is persistent (one CTA per SM), units are handed out round-robin in heaviest-first
-//     order (causal: last query tiles first), and every barrier phase carries across units.
+//     operand from TMEM: shared memory holds only Q_A, Q_B and a 4-stage K/V ring, and the tensor
+//     core reads half as many operand bytes from shared memory as with P in shared memory (also
+//     measured: an SS-operand P.V made the kernel shared-memory-bandwidth bound);
+//   * the grid is persistent (one CTA per SM), units are handed out round-robin batch by batch in
+//     heaviest-first order (causal: last query tiles first), and every barrier phase carries
+//     across units.
 // Warps: 0-7 softmax, 8 TMA producer, 9 TMEM allocator + MMA issuer.
 #pragma once
 
@@ -30,6 +38,13 @@ struct Prefill2Params {
   int causal;
   float scale_log2;
 };
+
+#ifndef ATTN_EXP2_EMULATE_MASK
+#define ATTN_EXP2_EMULATE_MASK 0x8888u
+#endif
+// Key pairs e (0..15 within each group of 32 keys) whose exponentials are computed with the FMA
+// polynomial (bit e set) instead of ex2.approx on the MUFU unit.
+constexpr uint32_t kExp2EmulateMask = ATTN_EXP2_EMULATE_MASK;
 
 template <int D>
 struct Prefill2Cfg {
@@ -68,13 +83,18 @@ struct UnitCoords {
   int b, h, q0;
 };
 
+// Unit order: batch-major, then heaviest (last) query-tile pairs first, then heads. CTAs take
+// units round-robin, so the units in flight at any time belong to one or two batches and share
+// their K/V in L2 (ordering heaviest-first across all batches made every batch's K/V live at once
+// and doubled the DRAM reads of a 16-batch prefill); within a batch the light causal pairs come
+// last, which keeps the tail short.
 __device__ __forceinline__ UnitCoords prefill_unit(const Prefill2Params& p, int u) {
-  const int BH = p.B * p.Hq;
-  const int i = u / BH, bh = u % BH;
+  const int per_batch = p.n_pairs * p.Hq;
+  const int rem = u % per_batch;
   UnitCoords c;
-  c.b = bh / p.Hq;
-  c.h = bh % p.Hq;
-  c.q0 = (p.n_pairs - 1 - i) * 256;  // heaviest (last) pairs first
+  c.b = u / per_batch;
+  c.h = rem % p.Hq;  // sibling query heads of a kv head are adjacent
+  c.q0 = (p.n_pairs - 1 - rem / p.Hq) * 256;
   return c;
 }
 
@@ -328,9 +348,16 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t xv = ffma2(f2_pack(s[q4][2 * e], s[q4][2 * e + 1]), c2x2, nm2);
-            float x0, x1;
-            f2_unpack(xv, x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            float p0, p1;
+            if (kExp2EmulateMask & (1u << e)) {
+              // this pair on the FMA pipe: the MUFU unit is the softmax's busiest resource
+              f2_unpack(exp2_poly2(xv), p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(xv, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             if (e & 1) acc1 = fadd2(acc1, f2_pack(p0, p1));
             else acc0 = fadd2(acc0, f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);

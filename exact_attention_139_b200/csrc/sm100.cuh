@@ -346,11 +346,45 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a pair of floats on the FMA pipe (x <= 64; relative error below 1e-4 for x >= -125;
+// inputs below -125 give values under 2^-124 instead of their exact subnormal value or 0). Range reduction to nearest: t = x + 1.5 * 2^23 holds n = round(x) in
+// its low mantissa bits, f = x - n lies in [-0.5, 0.5]; 2^f is the degree-3 polynomial with the
+// least maximum relative error on that interval, fitted by the Remez exchange algorithm
+// (exact_attention_139_b200/exp2_poly_fit.py; max relative error 7.5e-5 in fp32), and n is
+// added to the result's exponent field.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundShifter = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t xv);
+
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t xv) {
+  float x0, x1;
+  f2_unpack(xv, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xc, f2_pack(kRoundShifter, kRoundShifter));
+  const uint64_t n = fadd2(t, f2_pack(-kRoundShifter, -kRoundShifter));
+  const uint64_t f = ffma2(n, f2_pack(-1.f, -1.f), xc);  // x - n
+  uint64_t pp = ffma2(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  pp = ffma2(pp, f, f2_pack(kExp2C1, kExp2C1));
+  pp = ffma2(pp, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(pp, p0, p1);
+  f2_unpack(t, t0, t1);
+  // bits(t) = bits(1.5 * 2^23) + n and bits(1.5 * 2^23) << 23 == 0 (mod 2^32), so (bits(t) << 23)
+  // is n in the exponent field
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return f2_pack(r0, r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

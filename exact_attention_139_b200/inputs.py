@@ -15,6 +15,9 @@ Workloads (the shapes of the pages' settings; no dataset or model weights are us
     summary, "Planteamiento del Problema" and "Limitaciones").
   * ``long_prefill_128k``: B=1, Hq=32, Hkv=8, L=131072, causal, K biased by +2.0 on 64 random
     key positions per KV head (the vertical-column pattern of the MInference article).
+  * ``gqa_decode_32k``: GQA decode with a dense V, B=16, Hq=32, Hkv=8, Lq=1, Lk=32768,
+    d=dv=128 (the batch 8-16 regime of the "Flash Attention en Modelos Pequenos" notes on the
+    Llama-3-8B head shape).
 """
 from __future__ import annotations
 
@@ -86,6 +89,8 @@ WORKLOADS = {
                                latent=True, seed=BASE_SEED + 4),
     "long_prefill_128k": Workload("long_prefill_128k", 1, 32, 8, 131072, 131072, 128, 128, True,
                                   vertical_keys=64, vertical_bias=2.0, seed=BASE_SEED + 5),
+    "gqa_decode_32k": Workload("gqa_decode_32k", 16, 32, 8, 1, 32768, 128, 128, True,
+                               seed=BASE_SEED + 6),
 }
 
 

@@ -65,7 +65,8 @@ typedef enum {
  *   scale   multiplies Q.K^T (usually 1/sqrt(d)); must be finite and > 0.
  *   causal  0 = full attention, non-zero = bottom-right causal mask.
  * Supported: d == dv, d in {64, 128}; any B, Hq, Hkv (Hq % Hkv == 0), Lq, Lk >= 1.
- * Kernel: warp-specialised tcgen05/TMEM kernel with TMA loads (one CTA per 128-row Q tile).
+ * Kernel: persistent warp-specialised tcgen05/TMEM kernel with TMA loads; two 128-row query
+ * tiles per CTA ping-pong between two softmax warpgroups and one MMA-issuing thread.
  * Alignment: q, k, v, o 16-byte aligned (row strides are multiples of 16 bytes by shape).
  */
 attn_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
@@ -95,11 +96,13 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv
  *   workspace   device buffer of at least attn_decode_workspace_size(...) bytes, 256-byte
  *               aligned. Its contents on entry do not matter.
  * Supported: rows per kv head R = (Hq/Hkv)*Lq <= 64; d <= 576, dv <= 512, d and dv
- * multiples of 8 (16-byte rows). Two tensor-core kernels serve latent KV (v == k, ldv == d)
- * with d % 64 == 0, dv % 128 == 0, dv <= d and R <= 32: one puts the key length on the MMA M
- * dimension (the transposed flow of the FlashMLA-ETAP summary, "Mecanismo Central", items 1-3),
- * the other puts the query rows on M (padded to 64) and keys on N; attn_decode uses the one
- * measured faster on B200. Other shapes use a CUDA-core kernel.
+ * multiples of 8 (16-byte rows). Two tensor-core kernels serve R <= 32:
+ *   - query rows on the MMA M dimension (padded to 64), keys on N: latent KV (v == k, ldv == d,
+ *     d % 64 == 0, dv % 128 == 0, dv <= d) or a dense V with dv == d in {128, 256}; this is the
+ *     kernel attn_decode uses (measured fastest on B200);
+ *   - key length on M (the transposed flow of the FlashMLA-ETAP summary, "Mecanismo Central",
+ *     items 1-3): latent KV only, selectable through attn_decode_ex.
+ * Other shapes use a CUDA-core kernel.
  */
 attn_status attn_decode(const void *q, const void *k, const void *v, void *o, float *lse,
                         int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
@@ -177,6 +180,15 @@ attn_status attn_check_device(void *stream);
  * status. Enqueued on `stream`; returns ATTN_ERR_INVALID_ARG for a limit outside the range.
  */
 attn_status attn_selftest_wait_timeout(unsigned int limit_us, void *stream);
+
+/*
+ * attn_selftest_exp2 -- diagnostic: y[i] = 2^x[i] for n device floats, computed with the FMA-pipe
+ * polynomial the prefill softmax uses for part of its exponentials (round-to-nearest range
+ * reduction, degree-3 minimax polynomial; relative error below 1e-4 for x in [-125, 64]; below -125 the results are
+ * under 2^-124 but not accurate).
+ * x and y are device pointers; enqueued on `stream`.
+ */
+attn_status attn_selftest_exp2(const float *x, float *y, int n, void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *attn_status_string(attn_status status);

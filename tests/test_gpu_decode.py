@@ -35,6 +35,16 @@ def test_mla_decode_64k(impl, cuda_device):
     compare(og, lg, o_ref, l_ref, f"mla impl={impl}")
 
 
+@pytest.mark.parametrize("impl", [TN, CC])
+def test_gqa_decode_32k(impl, cuda_device):
+    """GQA decode with a dense V (16 x 32 query heads on 8 kv heads, 32K keys): every row."""
+    w = WORKLOADS["gqa_decode_32k"]
+    q, k, v, o, lse = run(w, cuda_device, impl=impl)
+    rows = np.arange(w.B * w.Hq * w.Lq)
+    o_ref, l_ref = oracle_rows(w, q, k, v, rows)
+    compare(o.reshape(-1, w.dv), lse.reshape(-1), o_ref, l_ref, f"gqa impl={impl}")
+
+
 SMALL = [
     # B, Hq, Hkv, Lq, Lk, d, dv, latent, causal
     (2, 16, 1, 2, 1000, 576, 512, True, True),
@@ -45,6 +55,8 @@ SMALL = [
     (1, 4, 4, 2, 65, 64, 64, False, True),
     (2, 32, 8, 2, 1500, 128, 128, False, True),
     (1, 8, 1, 1, 3, 128, 128, True, True),
+    (3, 16, 2, 2, 1000, 256, 256, False, True),
+    (2, 32, 1, 1, 4000, 128, 128, False, True),
 ]
 
 
@@ -58,8 +70,11 @@ def test_small_shapes(shape, splits, cuda_device):
     rows = np.arange(B * Hq * Lq)
     o_ref, l_ref = oracle_rows(w, q, k, v, rows)
     impls = [CC]
-    if latent and d % 64 == 0 and dv % 128 == 0 and (Hq // Hkv) * Lq <= 32:
+    R = (Hq // Hkv) * Lq
+    if latent and d % 64 == 0 and dv % 128 == 0 and R <= 32:
         impls += [TC, TN]
+    if not latent and dv == d and d in (128, 256) and R <= 32:
+        impls += [TN]
     qd, kd = q.to(cuda_device), k.to(cuda_device)
     vd = kd if latent else v.to(cuda_device)
     for impl in impls:
