@@ -5,8 +5,10 @@
 One step = one pass of the hot path over one batch of synthetic input. The default workload is the
 Llama-3-8B-shaped causal GQA prefill (B=1, Hq=32, Hkv=8, L=8192, d=128): metric attention TFLOPS
 (algorithmic flops = 2*(d+dv) per visible query/key pair). The same JSON line also carries the
-MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) measured in
-HBM GB/s, each with its roofline fraction against MEASURED_PEAKS.json.
+MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) and the GQA
+decode (B=16, 32 query heads on 8 kv heads, Lk=32768) measured in HBM GB/s, and the fp16-input
+variants of the prefill and of the MLA decode, each with its roofline fraction against
+MEASURED_PEAKS.json.
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching stream;
 L2 is flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU (torchrun):
@@ -194,7 +196,7 @@ def bench_prefill(w, dev, steps, warmup, flush, stream):
     from exact_attention_139_b200 import attn
     q, k, v = make_inputs(w)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=w.torch_dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
     step = lambda: attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
     times = time_steps(step, steps, warmup, flush, stream)
@@ -221,7 +223,7 @@ def bench_prefill_e2e(w, dev, steps, warmup, host):
     torch.cuda.synchronize()
     ms = start.elapsed_time(end) / steps
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-    d2h = bufs["o_host"].numel() * 2 + bufs["lse_host"].numel() * 4
+    d2h = bufs["o_host"].numel() * bufs["o_host"].element_size() + bufs["lse_host"].numel() * 4
     return ms, h2d, d2h
 
 
@@ -234,7 +236,7 @@ def bench_decode(w, dev, steps, warmup, flush, stream):
     splits = attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv)
     ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, splits),
                      dtype=torch.uint8, device=dev)
-    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=w.torch_dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
     step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=splits,
                                     workspace=ws, out=o, lse=lse)
@@ -310,6 +312,29 @@ def run_ours(args):
                          "note": "step = split kernel + combine kernel"},
             "tflops": round(wd.flops() / (dms * 1e-3) / 1e12, 1), "clocks": dclk}
         launches += 2 * args.steps
+        if not args.no_f16:
+            # fp16 inputs: same kernels with the fp16 operand format; fp16 and bf16 share one
+            # nominal tensor rate on B200, so the measured bf16 peak is the fp16 denominator
+            wf = rank_workload(WORKLOADS[args.workload].with_(dtype="f16"), rank)
+            ftimes, _ = bench_prefill(wf, dev, args.steps, args.warmup, flush, stream)
+            fms = max_over_ranks(sum(ftimes) / len(ftimes), world)
+            ftf = wf.flops() / (fms * 1e-3) / 1e12
+            extras["prefill_f16"] = {
+                "workload": wf.name + " (fp16 inputs)", "metric": "attention TFLOPS", "value": round(ftf * world, 2),
+                "ms_per_step": round(fms, 4),
+                "roofline": {"bound": "tensor", "achieved": round(ftf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": round(ftf / peak_tf, 4),
+                             "peak_source": f"{peak_src} bf16_tflops (burst) x 1 (fp16:bf16 nominal ratio)"}}
+            wdf = rank_workload(WORKLOADS["mla_decode_64k"].with_(dtype="f16"), rank)
+            dftimes, dfsplits = bench_decode(wdf, dev, args.steps, args.warmup, flush, stream)
+            dfms = max_over_ranks(sum(dftimes) / len(dftimes), world)
+            dfgbs = wdf.kv_bytes() / (dfms * 1e-3) / 1e9
+            extras["decode_f16"] = {
+                "workload": wdf.name + " (fp16 inputs)", "metric": "KV-read HBM GB/s", "value": round(dfgbs * world, 1),
+                "ms_per_step": round(dfms, 4), "num_splits": dfsplits,
+                "roofline": {"bound": "hbm", "achieved": round(dfgbs, 1), "peak": float(peaks["hbm_gbs"]),
+                             "unit": "GB/s", "frac": round(dfgbs / float(peaks["hbm_gbs"]), 4)}}
+            launches += args.steps + 2 * args.steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -331,7 +356,8 @@ def run_ours(args):
                          "frac": round(per_gpu_tflops / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "algorithmic_flops_per_launch": flops, "traffic": None},
             "e2e": e2e,
-            "gpu_launches": launches,
+            "gpu_launches": args.steps,  # one prefill kernel per timed step of the headline leg
+            "gpu_launches_all_legs": launches,
             "clocks": clk,
             "cpu_baseline": cpu,
             "extras": extras,
@@ -382,6 +408,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU (oracle) baseline")
     ap.add_argument("--no-extras", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--no-f16", action="store_true", help="skip the fp16-input measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

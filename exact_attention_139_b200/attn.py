@@ -4,10 +4,11 @@ Argument marshalling only: shapes are read from the torch tensors, device pointe
 current CUDA stream are passed through, and every step of the computation runs in the CUDA
 library. Importing this module raises if the library has not been built; there is no fallback.
 
-Functions keep the C names:
+Functions keep the C names; q, k, v (and o) are all bf16 or all fp16, and the element type is
+taken from q (the C ``*_typed`` entry points receive it):
     attn_fwd(q, k, v, causal=..., scale=None, out=None, lse=None)          -> (o, lse)
     attn_decode(q, k, v, causal=..., dv=None, num_splits=0, impl=0, ...)   -> (o, lse)
-    attn_combine(o_part, lse_part, out=None, lse=None)                     -> (o, lse)
+    attn_combine(o_part, lse_part, out=None, lse=None, dtype=bf16)         -> (o, lse)
     attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)         -> int
     attn_status_string(code), attn_check_device(), attn_selftest_wait_timeout(limit_us)
 plus attn_fwd_host(...): host tensors in, host tensors out (pinned copies around attn_fwd).
@@ -30,14 +31,20 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 
 _lib.attn_fwd.restype = _i
 _lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _vp]
+_lib.attn_fwd_typed.restype = _i
+_lib.attn_fwd_typed.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _i, _vp]
 _lib.attn_decode_workspace_size.restype = _sz
 _lib.attn_decode_workspace_size.argtypes = [_i] * 7
 _lib.attn_decode.restype = _i
 _lib.attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _sz, _vp]
 _lib.attn_decode_ex.restype = _i
 _lib.attn_decode_ex.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _sz, _i, _vp]
+_lib.attn_decode_typed.restype = _i
+_lib.attn_decode_typed.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _sz, _i, _i, _vp]
 _lib.attn_combine.restype = _i
 _lib.attn_combine.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp]
+_lib.attn_combine_typed.restype = _i
+_lib.attn_combine_typed.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp]
 _lib.attn_decode_default_splits.restype = _i
 _lib.attn_decode_default_splits.argtypes = [_i] * 7
 _lib.attn_check_device.restype = _i
@@ -52,6 +59,8 @@ _lib.attn_abi_version.argtypes = []
 ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED = 0, 1, 2, 3
 ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = 4, 5, 6
 ATTN_DECODE_AUTO, ATTN_DECODE_CUDA_CORE, ATTN_DECODE_TCGEN05_T, ATTN_DECODE_TCGEN05_N = 0, 1, 2, 3
+ATTN_DTYPE_BF16, ATTN_DTYPE_F16 = 0, 1
+_DTYPE_CODE = {torch.bfloat16: ATTN_DTYPE_BF16, torch.float16: ATTN_DTYPE_F16}
 
 
 class AttnError(RuntimeError):
@@ -90,22 +99,30 @@ def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _elem_code(q: torch.Tensor) -> int:
+    if q.dtype not in _DTYPE_CODE:
+        raise ValueError(f"q must be bfloat16 or float16, got {q.dtype}")
+    return _DTYPE_CODE[q.dtype]
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
              out: torch.Tensor | None = None, lse: torch.Tensor | None = None, want_lse: bool = True):
-    """O [B,Hq,Lq,dv] bf16 and LSE [B,Hq,Lq] fp32 for q [B,Hq,Lq,d], k/v [B,Hkv,Lk,d/dv]."""
+    """O [B,Hq,Lq,dv] (q's dtype) and LSE [B,Hq,Lq] fp32 for q [B,Hq,Lq,d], k/v [B,Hkv,Lk,d/dv]."""
+    code_t = _elem_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n)
+        _need(t, n, q.dtype)
     B, Hq, Lq, d = q.shape
     _, Hkv, Lk, _ = k.shape
     dv = v.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                         lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
-                         scale, int(bool(causal)), _stream_handle(q.device))
+    code = _lib.attn_fwd_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
+                               scale, int(bool(causal)), code_t, _stream_handle(q.device))
     _check(code, "attn_fwd")
     return out, lse
 
@@ -123,8 +140,9 @@ def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bo
                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
                 lse: torch.Tensor | None = None):
     """Split-KV decode. ``v is k`` selects the latent layout (V = first ``dv`` columns of K)."""
+    code_t = _elem_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n)
+        _need(t, n, q.dtype)
     B, Hq, Lq, d = q.shape
     _, Hkv, Lk, _ = k.shape
     ldv = v.shape[-1]
@@ -134,29 +152,34 @@ def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bo
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_decode_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                               B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, int(bool(causal)), int(num_splits),
-                               workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(impl),
-                               _stream_handle(q.device))
+    code = _lib.attn_decode_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, int(bool(causal)), int(num_splits),
+                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(impl),
+                                  code_t, _stream_handle(q.device))
     _check(code, "attn_decode")
     return out, lse
 
 
 def attn_combine(o_part: torch.Tensor, lse_part: torch.Tensor, *, B: int, Hq: int, Lq: int,
-                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
-    """o_part fp32 [S, B*Hq*Lq, dv], lse_part fp32 [S, B*Hq*Lq] -> O bf16 [B,Hq,Lq,dv], LSE."""
+                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                 dtype: torch.dtype = torch.bfloat16):
+    """o_part fp32 [S, B*Hq*Lq, dv], lse_part fp32 [S, B*Hq*Lq] -> O [B,Hq,Lq,dv] (``dtype``), LSE."""
     _need(o_part, "o_part", torch.float32)
     _need(lse_part, "lse_part", torch.float32)
+    if dtype not in _DTYPE_CODE:
+        raise ValueError(f"dtype must be bfloat16 or float16, got {dtype}")
     S, rows, dv = o_part.shape
     if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=o_part.device)
+        out = torch.empty((B, Hq, Lq, dv), dtype=dtype, device=o_part.device)
+    _need(out, "out", dtype)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=o_part.device)
-    code = _lib.attn_combine(o_part.data_ptr(), lse_part.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                             B, Hq, Lq, dv, S, _stream_handle(o_part.device))
+    code = _lib.attn_combine_typed(o_part.data_ptr(), lse_part.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                   B, Hq, Lq, dv, S, _DTYPE_CODE[dtype], _stream_handle(o_part.device))
     _check(code, "attn_combine")
     return out, lse
 
@@ -186,9 +209,9 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: 
             bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
         bufs[name].copy_(t, non_blocking=True)
     if "o" not in bufs:
-        bufs["o"] = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, device=dev)
+        bufs["o"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=dev)
         bufs["lse"] = torch.empty((B, Hq, Lq), dtype=torch.float32, device=dev)
-        bufs["o_host"] = torch.empty((B, Hq, Lq, dv), dtype=torch.bfloat16, pin_memory=True)
+        bufs["o_host"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, pin_memory=True)
         bufs["lse_host"] = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
     attn_fwd(bufs["q"], bufs["k"], bufs["v"], causal=causal, scale=scale, out=bufs["o"], lse=bufs["lse"])
     bufs["o_host"].copy_(bufs["o"], non_blocking=True)

@@ -21,7 +21,7 @@ namespace {
 
 using attn::DecodeParams;
 
-constexpr int kAbiVersion = 10000;  // 1.0.0
+constexpr int kAbiVersion = 10100;  // 1.1.0: element-type (*_typed) entry points
 
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -41,10 +41,11 @@ EncodeTiledFn get_encoder() {
   return fn;
 }
 
-// bf16 tensor map over a row-major [n2, n1, n0] array (n0 contiguous), 128-byte swizzle,
+// 16-bit-float tensor map over a row-major [n2, n1, n0] array (n0 contiguous), 128-byte swizzle,
 // zero fill out of bounds. box = {b0, b1, 1}. rank 2 when n2 == 0.
-bool encode_bf16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1,
-                 uint64_t row_stride = 0) {
+template <typename E>
+bool encode16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, uint64_t n2, uint32_t b0, uint32_t b1,
+              uint64_t row_stride = 0) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return false;
   const uint64_t rs = row_stride ? row_stride : n0;  // elements between consecutive rows
@@ -53,7 +54,7 @@ bool encode_bf16(CUtensorMap* map, const void* ptr, uint64_t n0, uint64_t n1, ui
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = n2 == 0 ? 2 : 3;
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+  CUresult r = enc(map, E::kFmt == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -154,43 +155,43 @@ int choose_splits(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int sms, int c
   return best;
 }
 
-template <int RMAX, int CPT>
+template <int RMAX, int CPT, typename E>
 attn_status launch_cc(const DecodeParams& p, int splits, cudaStream_t st) {
   const size_t smem = attn::decode_cc_smem_bytes(p.R, p.d, p.dv, !p.v_is_k);
-  auto kern = attn::decode_cc_kernel<RMAX, CPT>;
+  auto kern = attn::decode_cc_kernel<RMAX, CPT, E>;
   if (smem > 48 * 1024 && !allow_smem(kern, (int)smem)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
   kern<<<grid, attn::kCcThreads, smem, st>>>(p);
   return launch_status();
 }
 
-template <int DCH, int NB, int NP>
+template <int DCH, int NB, int NP, typename E>
 attn_status launch_tc(const DecodeParams& p, int splits, cudaStream_t st) {
   using C = attn::DecodeTcCfg<DCH, NB, NP>;
   CUtensorMap tq, tkv;
-  if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, NP)) return ATTN_ERR_CUDA;
-  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, C::BKV)) return ATTN_ERR_CUDA;
-  auto kern = attn::decode_tc_kernel<DCH, NB, NP>;
+  if (!encode16<E>(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, NP)) return ATTN_ERR_CUDA;
+  if (!encode16<E>(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, C::BKV)) return ATTN_ERR_CUDA;
+  auto kern = attn::decode_tc_kernel<DCH, NB, NP, E>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, p);
   return launch_status();
 }
 
-template <int DCH, int NB>
+template <int DCH, int NB, typename E>
 attn_status launch_tc_np(const DecodeParams& p, int splits, cudaStream_t st) {
-  if (p.R <= 16) return launch_tc<DCH, NB, 16>(p, splits, st);
-  return launch_tc<DCH, NB, 32>(p, splits, st);
+  if (p.R <= 16) return launch_tc<DCH, NB, 16, E>(p, splits, st);
+  return launch_tc<DCH, NB, 32, E>(p, splits, st);
 }
 
-template <int DCH>
+template <int DCH, typename E>
 attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
   switch (p.dv / 128) {
     // V^T block nb reads 64-column chunks 2nb and 2nb+1 of the latent tile, so 2*NB <= DCH
-    case 1: if constexpr (2 <= DCH) return launch_tc_np<DCH, 1>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
-    case 2: if constexpr (4 <= DCH) return launch_tc_np<DCH, 2>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
-    case 3: if constexpr (6 <= DCH) return launch_tc_np<DCH, 3>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
-    case 4: if constexpr (8 <= DCH) return launch_tc_np<DCH, 4>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 1: if constexpr (2 <= DCH) return launch_tc_np<DCH, 1, E>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 2: if constexpr (4 <= DCH) return launch_tc_np<DCH, 2, E>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 3: if constexpr (6 <= DCH) return launch_tc_np<DCH, 3, E>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
+    case 4: if constexpr (8 <= DCH) return launch_tc_np<DCH, 4, E>(p, splits, st); else return ATTN_ERR_UNSUPPORTED;
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
@@ -204,70 +205,73 @@ attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
 // Key tile and stage count of the queries-on-M decode kernel (chosen by measurement on B200).
 constexpr int kTnBK = ATTN_TN_BK, kTnNST = ATTN_TN_NST;
 
-template <int DCH, int NPIECE, int NST, bool SEPV>
+template <int DCH, int NPIECE, int NST, bool SEPV, typename E>
 attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
   using C = attn::DecodeTnCfg<DCH, NPIECE, kTnBK, NST, SEPV>;
   CUtensorMap tq, tkv, tv;
-  if (!encode_bf16(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
-  if (!encode_bf16(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK)) return ATTN_ERR_CUDA;
+  if (!encode16<E>(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
+  if (!encode16<E>(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK)) return ATTN_ERR_CUDA;
   if (SEPV) {
-    if (!encode_bf16(&tv, p.v, (uint64_t)p.dv, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK, (uint64_t)p.ldv))
+    if (!encode16<E>(&tv, p.v, (uint64_t)p.dv, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK, (uint64_t)p.ldv))
       return ATTN_ERR_CUDA;
   } else {
     tv = tkv;  // unused
   }
-  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, NST, SEPV>;
+  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, NST, SEPV, E>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, tv, p);
   return launch_status();
 }
 
-template <int DCH>
+template <int DCH, typename E>
 attn_status launch_tn_np(const DecodeParams& p, int splits, cudaStream_t st) {
-  if (p.dv <= 256) return launch_tn<DCH, 1, kTnNST, false>(p, splits, st);
-  return launch_tn<DCH, 2, kTnNST, false>(p, splits, st);
+  if (p.dv <= 256) return launch_tn<DCH, 1, kTnNST, false, E>(p, splits, st);
+  return launch_tn<DCH, 2, kTnNST, false, E>(p, splits, st);
 }
 
+template <typename E>
 attn_status launch_tn_any(const DecodeParams& p, int splits, cudaStream_t st) {
   if (!p.v_is_k) {
     // dense V beside K in each stage (small stages: a deeper ring)
-    if (p.d == 128) return launch_tn<2, 1, 6, true>(p, splits, st);
-    if (p.d == 256) return launch_tn<4, 1, 3, true>(p, splits, st);
+    if (p.d == 128) return launch_tn<2, 1, 6, true, E>(p, splits, st);
+    if (p.d == 256) return launch_tn<4, 1, 3, true, E>(p, splits, st);
     return ATTN_ERR_UNSUPPORTED;
   }
   switch (p.d / 64) {
-    case 2: return launch_tn_np<2>(p, splits, st);
-    case 3: return launch_tn_np<3>(p, splits, st);
-    case 4: return launch_tn_np<4>(p, splits, st);
-    case 5: return launch_tn_np<5>(p, splits, st);
-    case 6: return launch_tn_np<6>(p, splits, st);
-    case 7: return launch_tn_np<7>(p, splits, st);
-    case 8: return launch_tn_np<8>(p, splits, st);
-    case 9: return launch_tn_np<9>(p, splits, st);
+    case 2: return launch_tn_np<2, E>(p, splits, st);
+    case 3: return launch_tn_np<3, E>(p, splits, st);
+    case 4: return launch_tn_np<4, E>(p, splits, st);
+    case 5: return launch_tn_np<5, E>(p, splits, st);
+    case 6: return launch_tn_np<6, E>(p, splits, st);
+    case 7: return launch_tn_np<7, E>(p, splits, st);
+    case 8: return launch_tn_np<8, E>(p, splits, st);
+    case 9: return launch_tn_np<9, E>(p, splits, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
 
+template <typename E>
 attn_status launch_tc_any(const DecodeParams& p, int splits, cudaStream_t st) {
   switch (p.d / 64) {
-    case 2: return launch_tc_nb<2>(p, splits, st);
-    case 3: return launch_tc_nb<3>(p, splits, st);
-    case 4: return launch_tc_nb<4>(p, splits, st);
-    case 5: return launch_tc_nb<5>(p, splits, st);
-    case 6: return launch_tc_nb<6>(p, splits, st);
-    case 7: return launch_tc_nb<7>(p, splits, st);
-    case 8: return launch_tc_nb<8>(p, splits, st);
-    case 9: return launch_tc_nb<9>(p, splits, st);
+    case 2: return launch_tc_nb<2, E>(p, splits, st);
+    case 3: return launch_tc_nb<3, E>(p, splits, st);
+    case 4: return launch_tc_nb<4, E>(p, splits, st);
+    case 5: return launch_tc_nb<5, E>(p, splits, st);
+    case 6: return launch_tc_nb<6, E>(p, splits, st);
+    case 7: return launch_tc_nb<7, E>(p, splits, st);
+    case 8: return launch_tc_nb<8, E>(p, splits, st);
+    case 9: return launch_tc_nb<9, E>(p, splits, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
 
+template <typename E>
 attn_status launch_combine(const float* o_part, const float* lse_part, void* o, float* lse, long long rows, int dv,
                            int splits, cudaStream_t st) {
   if (rows <= 0) return ATTN_OK;
-  attn::combine_kernel<<<(unsigned)rows, attn::kCombineThreads, 0, st>>>(
-      o_part, lse_part, reinterpret_cast<__nv_bfloat16*>(o), lse, rows, dv, splits);
+  attn::combine_kernel<E><<<(unsigned)rows, attn::kCombineThreads, 0, st>>>(
+      o_part, lse_part, reinterpret_cast<uint16_t*>(o), lse, rows, dv, splits);
   return launch_status();
 }
 
@@ -303,37 +307,30 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restr
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-const char* attn_status_string(attn_status s) {
-  switch (s) {
-    case ATTN_OK: return "ok";
-    case ATTN_ERR_INVALID_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported shape";
-    case ATTN_ERR_MISALIGNED: return "misaligned pointer or stride";
-    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
-    case ATTN_ERR_CUDA: return "CUDA error";
-    case ATTN_ERR_TIMEOUT: return "a bounded wait on the GPU ran out";
-  }
-  return "unknown status";
+// --- typed entry points: dispatch on the element type ---
+bool valid_dtype(int dtype) { return dtype == ATTN_DTYPE_BF16 || dtype == ATTN_DTYPE_F16; }
+
+template <typename Fn>
+attn_status with_elem(int dtype, Fn&& fn) {
+  if (dtype == ATTN_DTYPE_BF16) return fn(attn::ElemBf16{});
+  if (dtype == ATTN_DTYPE_F16) return fn(attn::ElemF16{});
+  return ATTN_ERR_INVALID_ARG;
 }
 
-int attn_abi_version(void) { return kAbiVersion; }
-
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
-                     int Lk, int d, int dv, float scale, int causal, void* stream) {
-  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
-  if (st != ATTN_OK) return st;
-  if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+template <typename E>
+attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                     int Lk, int d, float scale, int causal, void* stream) {
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int n_qtiles = (Lq + 127) / 128;
   CUtensorMap tq, tk, tv;
-  if (!encode_bf16(&tq, q, (uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
-      !encode_bf16(&tk, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
-      !encode_bf16(&tv, v, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
+  if (!encode16<E>(&tq, q, (uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
+      !encode16<E>(&tk, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
+      !encode16<E>(&tv, v, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
     return ATTN_ERR_CUDA;
   attn::Prefill2Params p{};
-  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.o = reinterpret_cast<uint16_t*>(o);
   p.lse = lse;
   p.B = B;
   p.Hq = Hq;
@@ -351,32 +348,20 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   const int grid = (int)std::min<long long>(units, current_sm_count());
   if (d == 128) {
     using C = attn::Prefill2Cfg<128>;
-    if (!allow_smem(attn::prefill2_kernel<128>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<128><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    if (!allow_smem(attn::prefill2_kernel<128, E>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<128, E><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   } else {
     using C = attn::Prefill2Cfg<64>;
-    if (!allow_smem(attn::prefill2_kernel<64>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<64><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    if (!allow_smem(attn::prefill2_kernel<64, E>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<64, E><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   }
   return launch_status();
 }
 
-size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int num_splits) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || dv < 1 || num_splits < 0 || num_splits > 256) return 0;
-  if (Hq % Hkv != 0) return 0;
-  int s = num_splits;
-  if (s == 0) s = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
-  return workspace_bytes((long long)B * Hq * Lq, dv, s);
-}
-
-int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
-  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
-}
-
-attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                           int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
-                           void* workspace, size_t ws_bytes, int impl, void* stream) {
+template <typename E>
+attn_status decode_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                        void* workspace, size_t ws_bytes, int impl, void* stream) {
   attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
   if (st != ATTN_OK) return st;
   if (ldv < dv) return ATTN_ERR_INVALID_ARG;
@@ -397,9 +382,9 @@ attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o,
   if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
 
   DecodeParams p{};
-  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
-  p.k = reinterpret_cast<const __nv_bfloat16*>(k);
-  p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.q = reinterpret_cast<const uint16_t*>(q);
+  p.k = reinterpret_cast<const uint16_t*>(k);
+  p.v = reinterpret_cast<const uint16_t*>(v);
   p.o_part = reinterpret_cast<float*>(workspace);
   p.lse_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + align256((size_t)splits * rows * dv * 4));
   p.rows_total = rows;
@@ -420,17 +405,82 @@ attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o,
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   if (impl == ATTN_DECODE_TCGEN05_T) {
-    st = launch_tc_any(p, splits, cs);
+    st = launch_tc_any<E>(p, splits, cs);
   } else if (impl == ATTN_DECODE_TCGEN05_N) {
-    st = launch_tn_any(p, splits, cs);
+    st = launch_tn_any<E>(p, splits, cs);
   } else {
     const int cpt = (dv + attn::kCcThreads - 1) / attn::kCcThreads;
-    if (p.R <= 16) st = cpt == 1 ? launch_cc<16, 1>(p, splits, cs) : launch_cc<16, 2>(p, splits, cs);
-    else if (p.R <= 32) st = cpt == 1 ? launch_cc<32, 1>(p, splits, cs) : launch_cc<32, 2>(p, splits, cs);
-    else st = cpt == 1 ? launch_cc<64, 1>(p, splits, cs) : launch_cc<64, 2>(p, splits, cs);
+    if (p.R <= 16) st = cpt == 1 ? launch_cc<16, 1, E>(p, splits, cs) : launch_cc<16, 2, E>(p, splits, cs);
+    else if (p.R <= 32) st = cpt == 1 ? launch_cc<32, 1, E>(p, splits, cs) : launch_cc<32, 2, E>(p, splits, cs);
+    else st = cpt == 1 ? launch_cc<64, 1, E>(p, splits, cs) : launch_cc<64, 2, E>(p, splits, cs);
   }
   if (st != ATTN_OK) return st;
-  return launch_combine(p.o_part, p.lse_part, o, lse, rows, dv, splits, cs);
+  return launch_combine<E>(p.o_part, p.lse_part, o, lse, rows, dv, splits, cs);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case ATTN_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "a bounded wait on the GPU ran out";
+  }
+  return "unknown status";
+}
+
+int attn_abi_version(void) { return kAbiVersion; }
+
+attn_status attn_fwd_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Lq, int Lk, int d, int dv, float scale, int causal, int dtype, void* stream) {
+  if (!valid_dtype(dtype)) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+  return with_elem(dtype, [&](auto e) {
+    return fwd_impl<decltype(e)>(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal, stream);
+  });
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                     int Lk, int d, int dv, float scale, int causal, void* stream) {
+  return attn_fwd_typed(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal, ATTN_DTYPE_BF16, stream);
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || dv < 1 || num_splits < 0 || num_splits > 256) return 0;
+  if (Hq % Hkv != 0) return 0;
+  int s = num_splits;
+  if (s == 0) s = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  return workspace_bytes((long long)B * Hq * Lq, dv, s);
+}
+
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
+  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+}
+
+attn_status attn_decode_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                              int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                              void* workspace, size_t ws_bytes, int impl, int dtype, void* stream) {
+  if (!valid_dtype(dtype)) return ATTN_ERR_INVALID_ARG;
+  return with_elem(dtype, [&](auto e) {
+    return decode_impl<decltype(e)>(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits,
+                                    workspace, ws_bytes, impl, stream);
+  });
+}
+
+attn_status attn_decode_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                           void* workspace, size_t ws_bytes, int impl, void* stream) {
+  return attn_decode_typed(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits, workspace,
+                           ws_bytes, impl, ATTN_DTYPE_BF16, stream);
 }
 
 attn_status attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -490,8 +540,9 @@ attn_status attn_decode_noalloc(const void* q, const void* k, const void* v, voi
                         (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES, ATTN_DECODE_AUTO, stream);
 }
 
-attn_status attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq, int Lq,
-                         int dv, int num_splits, void* stream) {
+attn_status attn_combine_typed(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq,
+                               int Lq, int dv, int num_splits, int dtype, void* stream) {
+  if (!valid_dtype(dtype)) return ATTN_ERR_INVALID_ARG;
   if (!o_part || !lse_part || !o) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Lq < 1 || dv < 1 || num_splits < 1 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
   if (dv % 4 != 0) return ATTN_ERR_MISALIGNED;
@@ -499,7 +550,15 @@ attn_status attn_combine(const float* o_part, const float* lse_part, void* o, fl
     return ATTN_ERR_MISALIGNED;
   const long long rows = (long long)B * Hq * Lq;
   if (rows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  return launch_combine(o_part, lse_part, o, lse, rows, dv, num_splits, reinterpret_cast<cudaStream_t>(stream));
+  return with_elem(dtype, [&](auto e) {
+    return launch_combine<decltype(e)>(o_part, lse_part, o, lse, rows, dv, num_splits,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  });
+}
+
+attn_status attn_combine(const float* o_part, const float* lse_part, void* o, float* lse, int B, int Hq, int Lq,
+                         int dv, int num_splits, void* stream) {
+  return attn_combine_typed(o_part, lse_part, o, lse, B, Hq, Lq, dv, num_splits, ATTN_DTYPE_BF16, stream);
 }
 
 attn_status attn_selftest_wait_timeout(unsigned int limit_us, void* stream) {

@@ -12,9 +12,10 @@ namespace attn {
 
 constexpr int kCombineThreads = 128;
 
+template <typename E>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                   __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long rows, int dv,
+                   uint16_t* __restrict__ o, float* __restrict__ lse, long long rows, int dv,
                    int num_splits) {
   const long long row = blockIdx.x;
   float m = -INFINITY;
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(kCombineThreads)
         acc.w = fmaf(w, x.w, acc.w);
       }
     }
-    uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    uint2 packed = make_uint2(E::pack2(acc.x, acc.y), E::pack2(acc.z, acc.w));
     *reinterpret_cast<uint2*>(o + row * dv + c) = packed;
   }
   if (threadIdx.x == 0 && lse != nullptr) lse[row] = L;

@@ -21,9 +21,9 @@
 namespace attn {
 
 struct DecodeParams {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k;
-  const __nv_bfloat16* v;
+  const uint16_t* q;  // 16-bit floats of the kernel's element type
+  const uint16_t* k;
+  const uint16_t* v;
   float* o_part;    // [num_splits, rows_total, dv]
   float* lse_part;  // [num_splits, rows_total]
   long long rows_total;
@@ -51,7 +51,7 @@ __host__ inline size_t decode_cc_smem_bytes(int R, int d, int dv, bool separate_
   return b;
 }
 
-template <int RMAX, int CPT>
+template <int RMAX, int CPT, typename E>
 __global__ void __launch_bounds__(kCcThreads)
     decode_cc_kernel(const DecodeParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -63,9 +63,9 @@ __global__ void __launch_bounds__(kCcThreads)
   const int ks = cc_row_stride(p.d), vs = cc_row_stride(p.dv);
   const bool sep_v = !p.v_is_k;
 
-  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* Ks = Qs + (size_t)R * p.d;
-  __nv_bfloat16* Vs = Ks + (size_t)kCcKeys * ks;
+  uint16_t* Qs = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* Ks = Qs + (size_t)R * p.d;
+  uint16_t* Vs = Ks + (size_t)kCcKeys * ks;
   float* Ss = reinterpret_cast<float*>(Vs + (sep_v ? (size_t)kCcKeys * vs : 0));
   float* alpha_s = Ss + 64 * kCcKeys;
   float* l_s = alpha_s + 64;
@@ -88,8 +88,8 @@ __global__ void __launch_bounds__(kCcThreads)
     for (int cc = 0; cc < CPT; ++cc) acc[r][cc] = 0.f;
   float m_run = -INFINITY, l_run = 0.f;  // meaningful in threads tid < R
 
-  const __nv_bfloat16* kbase = p.k + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.d;
-  const __nv_bfloat16* vbase = p.v + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.ldv;
+  const uint16_t* kbase = p.k + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.d;
+  const uint16_t* vbase = p.v + ((long long)b * p.Hkv + hkv) * (long long)p.Lk * p.ldv;
 
   for (int kc = j_begin; kc < j_end; kc += kCcKeys) {
     __syncthreads();  // previous chunk fully consumed
@@ -116,12 +116,12 @@ __global__ void __launch_bounds__(kCcThreads)
       const int i = r % p.Lq;
       float sc = -INFINITY;
       if (jr < nk && (!p.causal || key <= i + off)) {
-        const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(Qs + r * p.d);
-        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(Ks + jr * ks);
+        const uint32_t* qr = reinterpret_cast<const uint32_t*>(Qs + r * p.d);
+        const uint32_t* kr = reinterpret_cast<const uint32_t*>(Ks + jr * ks);
         float a0 = 0.f, a1 = 0.f;
         for (int c = 0; c < p.d / 2; ++c) {
-          const float2 qf = __bfloat1622float2(qr[c]);
-          const float2 kf = __bfloat1622float2(kr[c]);
+          const float2 qf = E::unpack2(qr[c]);
+          const float2 kf = E::unpack2(kr[c]);
           a0 = fmaf(qf.x, kf.x, a0);
           a1 = fmaf(qf.y, kf.y, a1);
         }
@@ -158,14 +158,14 @@ __global__ void __launch_bounds__(kCcThreads)
         for (int cc = 0; cc < CPT; ++cc) acc[r][cc] *= a;
       }
     }
-    const __nv_bfloat16* Vsrc = sep_v ? Vs : Ks;
+    const uint16_t* Vsrc = sep_v ? Vs : Ks;
     const int vstride = sep_v ? vs : ks;
     for (int jr = 0; jr < nk; ++jr) {
       float vv[CPT];
 #pragma unroll
       for (int cc = 0; cc < CPT; ++cc) {
         const int c = tid + cc * kCcThreads;
-        vv[cc] = (c < p.dv) ? __bfloat162float(Vsrc[jr * vstride + c]) : 0.f;
+        vv[cc] = (c < p.dv) ? E::to_float(Vsrc[jr * vstride + c]) : 0.f;
       }
 #pragma unroll
       for (int r = 0; r < RMAX; ++r) {
@@ -267,7 +267,7 @@ __device__ __forceinline__ void tmem_st_np(uint32_t taddr, const float (&v)[32])
   }
 }
 
-template <int DCH, int NB, int NP>
+template <int DCH, int NB, int NP, typename E>
 __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                      const DecodeParams p) {
@@ -352,8 +352,8 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
   } else if (warp == 5) {
     // ------------------------------- MMA issuer -------------------------------
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(64, NP, false, false);  // S^T = K.Q^T
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, NP, true, false);  // O^T += V^T.P^T
+      constexpr uint32_t idesc_s = make_idesc(64, NP, false, false, E::kFmt);  // S^T = K.Q^T
+      constexpr uint32_t idesc_o = make_idesc(128, NP, true, false, E::kFmt);  // O^T += V^T.P^T
       bool ok = mbar_wait(bar_q, 0, 22);
       bool issued = false;
       auto pv = [&](int tt) {
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
           // element (n, key kr) of the K-major no-swizzle P^T tile
           const uint32_t o = (uint32_t)(n >> 3) * 1024u + (uint32_t)(kr >> 3) * 128u +
                              (uint32_t)(n & 7) * 16u + (uint32_t)(kr & 7) * 2u;
-          *reinterpret_cast<__nv_bfloat16*>(pbuf + o) = __float2bfloat16_rn(pr);
+          *reinterpret_cast<uint16_t*>(pbuf + o) = (uint16_t)(E::pack2(pr, 0.f) & 0xFFFFu);
         }
       }
       ok = group_sync();
@@ -630,7 +630,7 @@ __device__ __forceinline__ void tmem_ld_keys(uint32_t taddr, float (&x)[64]) {
   }
 }
 
-template <int DCH, int NPIECE, int BK, int NST, bool SEPV>
+template <int DCH, int NPIECE, int BK, int NST, bool SEPV, typename E>
 __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREADS, 1)
     decode_tn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -721,7 +721,7 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
   } else if (warp >= 4) {
     // -------------------- S issuers: partial a = chunks a, a + NACC, ... --------------------
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(64, BK, false, false);  // S = Q.K^T
+      constexpr uint32_t idesc_s = make_idesc(64, BK, false, false, E::kFmt);  // S = Q.K^T
       const int a = warp - 4;
       const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL + a * BK;
       const uint64_t qdesc = make_sdesc(base + C::OFF_Q + a * C::QCH, 16, 1024, kSwizzle128B);
@@ -756,7 +756,7 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
   } else if (warp == 3) {
     // ------------------------------- P.V issuer -------------------------------
     if (lane == 0 && n_tiles > 0) {
-      const uint32_t idesc_o = make_idesc_bf16(64, NW, false, true);  // O += P.V
+      const uint32_t idesc_o = make_idesc(64, NW, false, true, E::kFmt);  // O += P.V
       bool ok = true, issued = false;
       for (int t = 0; t < n_tiles && ok; ++t) {
         ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
@@ -848,7 +848,7 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
           const float p0 = ex2_approx(fmaf(x[8 * u + 2 * e], c2, -m_ref));
           const float p1 = ex2_approx(fmaf(x[8 * u + 2 * e + 1], c2, -m_ref));
           sum += p0 + p1;
-          w4[e] = pack_bf16x2(p0, p1);
+          w4[e] = E::pack2(p0, p1);
         }
         if (s_lane)
           *reinterpret_cast<uint4*>(prow + swz128_offset((uint32_t)m, (uint32_t)u)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);

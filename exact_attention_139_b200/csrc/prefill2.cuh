@@ -30,7 +30,7 @@
 namespace attn {
 
 struct Prefill2Params {
-  __nv_bfloat16* o;
+  uint16_t* o;  // 16-bit floats of the kernel's element type
   float* lse;
   int B, Hq, Hkv, Lq, Lk, G;
   int n_pairs;  // ceil(ceil(Lq / 128) / 2)
@@ -98,7 +98,7 @@ __device__ __forceinline__ UnitCoords prefill_unit(const Prefill2Params& p, int 
   return c;
 }
 
-template <int D>
+template <int D, typename E>
 __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Prefill2Params p) {
@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
   } else if (warp == 9) {
     // ------------------------------- MMA issuer -------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(C::BM, C::BN, false, false);
-      constexpr uint32_t idesc_o = make_idesc_bf16(C::BM, D, false, true);
+      constexpr uint32_t idesc_s = make_idesc(C::BM, C::BN, false, false, E::kFmt);
+      constexpr uint32_t idesc_o = make_idesc(C::BM, D, false, true, E::kFmt);
       bool ok = true, issued = false;
       int kv_t = 0, qc = 0;
       int p_cnt[2] = {0, 0}, units_done[2] = {0, 0};
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             }
             if (e & 1) acc1 = fadd2(acc1, f2_pack(p0, p1));
             else acc0 = fadd2(acc0, f2_pack(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
+            pk[e] = E::pack2(p0, p1);
           }
           // P overwrites the S columns it came from: keys 32*q4 .. 32*q4 + 31
           tmem_st16u(tw + s_col + 16 * q4, pk);
@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool in_range = row < p.Lq;
-      __nv_bfloat16* orow = p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + (in_range ? row : 0)) * D;
+      uint16_t* orow = p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + (in_range ? row : 0)) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         float o[32];
@@ -405,10 +405,10 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16x2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l),
-                                pack_bf16x2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l),
-                                pack_bf16x2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l),
-                                pack_bf16x2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
+            dst[q] = make_uint4(E::pack2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l),
+                                E::pack2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l),
+                                E::pack2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l),
+                                E::pack2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
         }
       }
       if (in_range && p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = (m_used + log2f(l)) * kLn2;

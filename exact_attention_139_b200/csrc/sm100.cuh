@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace attn {
@@ -226,16 +227,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 // ---------------------------------------------------------------------------------------
 // tcgen05: MMA (kind::f16 with bf16 operands, fp32 accumulator in TMEM)
 // ---------------------------------------------------------------------------------------
-// Instruction descriptor: D fp32, A and B bf16, dense, no negation; a_mn / b_mn select the
-// MN-major (transposed) operand layout; N in units of 8, M in units of 16.
-__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+// Instruction descriptor: D fp32, A and B 16-bit floats of format `fmt` (0 fp16, 1 bf16), dense,
+// no negation; a_mn / b_mn select the MN-major (transposed) operand layout; N in units of 8, M in
+// units of 16.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool a_mn, bool b_mn, uint32_t fmt) {
   return (1u << 4)                               // D format: f32
-         | (1u << 7)                             // A format: bf16
-         | (1u << 10)                            // B format: bf16
+         | (fmt << 7)                            // A format
+         | (fmt << 10)                           // B format
          | ((a_mn ? 1u : 0u) << 15)              // A major
          | ((b_mn ? 1u : 0u) << 16)              // B major
          | ((uint32_t)(N >> 3) << 17)            // N >> 3
          | ((uint32_t)(M >> 4) << 24);           // M >> 4
+}
+
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return make_idesc(M, N, a_mn, b_mn, 1u);
 }
 
 // Shared-memory matrix descriptor (sm_100 version bit set).
@@ -289,6 +295,25 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
       "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
+}
+
+// 32 lanes x 32 bits, 8 consecutive columns (load and store).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
 }
 
 // 32 lanes x 32 bits, 16 consecutive columns from raw 32-bit words.
@@ -391,6 +416,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+
+// Element type of Q, K, V, P and O: bf16 or fp16 (both tcgen05 kind::f16; only the operand
+// format code, the conversions and the TMA data type differ).
+struct ElemBf16 {
+  static constexpr uint32_t kFmt = 1;
+  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  __device__ __forceinline__ static float2 unpack2(uint32_t w) {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w);
+    return __bfloat1622float2(h);
+  }
+  __device__ __forceinline__ static float to_float(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
+};
+
+struct ElemF16 {
+  static constexpr uint32_t kFmt = 0;
+  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ __forceinline__ static float2 unpack2(uint32_t w) {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    return __half22float2(h);
+  }
+  __device__ __forceinline__ static float to_float(uint16_t x) { return __half2float(__ushort_as_half(x)); }
+};
 
 // Byte offset of 16-byte unit `u` of row `r` in a 128-byte-swizzled tile (rows of 128 B,
 // 1024-byte aligned base): the unit index is XORed with the row index modulo 8.

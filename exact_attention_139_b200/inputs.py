@@ -1,7 +1,8 @@
 """Seeded synthetic inputs shared by the CUDA path's tests/benchmark and the oracle's tests.
 
 This module holds no attention arithmetic: it only draws N(0, 1) values, adds the optional
-'vertical' key bias and rounds once to bf16. Everything is generated on the CPU with a seeded
+'vertical' key bias and rounds once to the workload's 16-bit type (bf16, or fp16 for the
+``*_f16`` variants made with ``with_(dtype="f16")``). Everything is generated on the CPU with a seeded
 ``torch.Generator`` so both sides see the same bits.
 
 Workloads (the shapes of the pages' settings; no dataset or model weights are used):
@@ -44,6 +45,11 @@ class Workload:
     vertical_keys: int = 0        # number of biased key positions per KV head
     vertical_bias: float = 0.0
     seed: int = BASE_SEED
+    dtype: str = "bf16"           # element type of q, k, v and o: "bf16" or "f16"
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return {"bf16": torch.bfloat16, "f16": torch.float16}[self.dtype]
 
     @property
     def scale(self) -> float:
@@ -94,41 +100,43 @@ WORKLOADS = {
 }
 
 
-def _planes(g: torch.Generator, lead: int, rows: int, cols: int) -> torch.Tensor:
-    """lead x rows x cols bf16 values, drawn plane by plane as fp32 N(0,1), rounded once."""
-    out = torch.empty((lead, rows, cols), dtype=torch.bfloat16)
+def _planes(g: torch.Generator, lead: int, rows: int, cols: int, dtype=torch.bfloat16) -> torch.Tensor:
+    """lead x rows x cols 16-bit values, drawn plane by plane as fp32 N(0,1), rounded once."""
+    out = torch.empty((lead, rows, cols), dtype=dtype)
     for p in range(lead):
-        out[p] = torch.randn((rows, cols), generator=g, dtype=torch.float32).to(torch.bfloat16)
+        out[p] = torch.randn((rows, cols), generator=g, dtype=torch.float32).to(dtype)
     return out
 
 
 def make_inputs(w: Workload):
-    """(q, k, v) bf16 CPU tensors for workload ``w``; v is k itself for latent workloads.
+    """(q, k, v) CPU tensors of ``w.torch_dtype`` for workload ``w``; v is k itself for latent
+    workloads. The fp16 variant draws the same fp32 values as the bf16 one.
 
     Draw order: Q planes, K planes, V planes (each (b, h) plane in order), then the biased key
     positions (one ``randperm`` per (b, kv head)). The bias is added to the fp32 draw before the
     single rounding to bf16, so K is regenerated plane by plane when a bias is requested.
     """
     g = torch.Generator().manual_seed(w.seed)
-    q = _planes(g, w.B * w.Hq, w.Lq, w.d).view(w.B, w.Hq, w.Lq, w.d)
+    dt = w.torch_dtype
+    q = _planes(g, w.B * w.Hq, w.Lq, w.d, dt).view(w.B, w.Hq, w.Lq, w.d)
     if w.vertical_keys == 0:
-        k = _planes(g, w.B * w.Hkv, w.Lk, w.d).view(w.B, w.Hkv, w.Lk, w.d)
-        v = k if w.latent else _planes(g, w.B * w.Hkv, w.Lk, w.dv).view(w.B, w.Hkv, w.Lk, w.dv)
+        k = _planes(g, w.B * w.Hkv, w.Lk, w.d, dt).view(w.B, w.Hkv, w.Lk, w.d)
+        v = k if w.latent else _planes(g, w.B * w.Hkv, w.Lk, w.dv, dt).view(w.B, w.Hkv, w.Lk, w.dv)
         return q, k, v
     # keep the fp32 K draw (one plane at a time) until the positions are known
     kstate = g.get_state()
     for _ in range(w.B * w.Hkv):
         torch.randn((w.Lk, w.d), generator=g, dtype=torch.float32)
-    v = None if w.latent else _planes(g, w.B * w.Hkv, w.Lk, w.dv).view(w.B, w.Hkv, w.Lk, w.dv)
+    v = None if w.latent else _planes(g, w.B * w.Hkv, w.Lk, w.dv, dt).view(w.B, w.Hkv, w.Lk, w.dv)
     positions = [torch.randperm(w.Lk, generator=g)[: w.vertical_keys]
                  for _ in range(w.B * w.Hkv)]
     g2 = torch.Generator()
     g2.set_state(kstate)
-    k = torch.empty((w.B * w.Hkv, w.Lk, w.d), dtype=torch.bfloat16)
+    k = torch.empty((w.B * w.Hkv, w.Lk, w.d), dtype=dt)
     for p in range(w.B * w.Hkv):
         plane = torch.randn((w.Lk, w.d), generator=g2, dtype=torch.float32)
         plane[positions[p]] += w.vertical_bias
-        k[p] = plane.to(torch.bfloat16)
+        k[p] = plane.to(dt)
     k = k.view(w.B, w.Hkv, w.Lk, w.d)
     return q, k, (k if w.latent else v)
 

@@ -18,18 +18,19 @@
  *    soon as the work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *    default stream).
  *  - Layouts are row-major and contiguous:
- *        q   [B, Hq,  Lq, d]   bf16
- *        k   [B, Hkv, Lk, d]   bf16
- *        v   [B, Hkv, Lk, ldv] bf16, the first dv columns of each row are used
- *        o   [B, Hq,  Lq, dv]  bf16
+ *        q   [B, Hq,  Lq, d]   bf16 (or fp16, see the *_typed entry points)
+ *        k   [B, Hkv, Lk, d]   same element type as q
+ *        v   [B, Hkv, Lk, ldv] same element type, the first dv columns of each row are used
+ *        o   [B, Hq,  Lq, dv]  same element type
  *        lse [B, Hq,  Lq]      fp32 (may be NULL)
  *  - GQA: query head h reads kv head h / (Hq / Hkv); Hq must be a multiple of Hkv.
  *  - Causal masking is bottom-right aligned: key j is visible to query row i iff
  *    j <= i + (Lk - Lq), i.e. the Lq queries are the last Lq positions of the sequence.
  *    causal != 0 with Lq > Lk is rejected (some rows would see no key).
  *  - LSE is the natural logarithm of sum_j exp(scale * q_i . k_j) over the visible keys.
- *  - Arithmetic: bf16 inputs, fp32 accumulation on the tensor cores, fp32 softmax, P rounded
- *    to bf16 before P.V, O rounded to bf16 (round-to-nearest-even) at the end.
+ *  - Arithmetic: 16-bit inputs (bf16 by default), fp32 accumulation on the tensor cores, fp32
+ *    softmax, P rounded to the input type before P.V, O rounded to the input type
+ *    (round-to-nearest-even) at the end.
  *  - Errors: argument checks run on the host before any launch and return a non-zero status
  *    with nothing enqueued. A failed launch returns ATTN_ERR_CUDA. Kernels bound every wait
  *    on the GPU; a wait that runs out records ATTN_ERR_TIMEOUT in a device-side word that
@@ -58,6 +59,19 @@ typedef enum {
 } attn_status;
 
 /*
+ * Element type of q, k, v and o for the *_typed entry points. The untyped entry points take
+ * bf16. FP16 is the input type of the FlashMLA-ETAP summary's measurements (H20, 148 TFLOPS
+ * FP16, "Planteamiento del Problema"); both types run the same kernels, only the tensor-core
+ * operand format, the TMA element type and the rounding of P and O change. FP16 keeps 10
+ * mantissa bits but overflows above 65504: P lies in [0, 1] and O is a convex combination of V
+ * rows, so neither can overflow when q, k and v are finite fp16 values.
+ */
+typedef enum {
+    ATTN_DTYPE_BF16 = 0,
+    ATTN_DTYPE_F16 = 1
+} attn_dtype;
+
+/*
  * attn_fwd -- prefill / general forward attention.
  *
  * Computes O and (optionally) LSE for all B*Hq*Lq query rows against Lk keys. V is dense:
@@ -72,6 +86,11 @@ typedef enum {
 attn_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                      int Hq, int Hkv, int Lq, int Lk, int d, int dv, float scale, int causal,
                      void *stream);
+
+/* attn_fwd for element type `dtype` (an attn_dtype); ATTN_ERR_INVALID_ARG for another value. */
+attn_status attn_fwd_typed(const void *q, const void *k, const void *v, void *o, float *lse,
+                           int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, float scale,
+                           int causal, int dtype, void *stream);
 
 /*
  * attn_decode_workspace_size -- bytes of device workspace attn_decode needs for the given
@@ -124,6 +143,13 @@ attn_status attn_decode_ex(const void *q, const void *k, const void *v, void *o,
                            float scale, int causal, int num_splits, void *workspace,
                            size_t workspace_bytes, int impl, void *stream);
 
+/* attn_decode_ex for element type `dtype` (an attn_dtype); ATTN_ERR_INVALID_ARG for another
+ * value. The workspace partials are fp32 whatever the element type. */
+attn_status attn_decode_typed(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int ldv,
+                              float scale, int causal, int num_splits, void *workspace,
+                              size_t workspace_bytes, int impl, int dtype, void *stream);
+
 /*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
  *
@@ -160,6 +186,11 @@ attn_status attn_decode_noalloc(const void *q, const void *k, const void *v, voi
  */
 attn_status attn_combine(const float *o_part, const float *lse_part, void *o, float *lse,
                          int B, int Hq, int Lq, int dv, int num_splits, void *stream);
+
+/* attn_combine writing o in element type `dtype` (an attn_dtype). */
+attn_status attn_combine_typed(const float *o_part, const float *lse_part, void *o, float *lse,
+                               int B, int Hq, int Lq, int dv, int num_splits, int dtype,
+                               void *stream);
 
 /* Number of splits attn_decode would choose (num_splits = 0) on the current device. */
 int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv);

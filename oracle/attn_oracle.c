@@ -31,7 +31,9 @@
  *   - LSE is the natural log of sum_j exp(s_ij) over the visible keys, scale included;
  *   - an empty visible set gives O = 0 and LSE = -inf (this only occurs for split
  *     partials, never for a whole row, because causal calls need Lq <= Lk);
- *   - inputs are bf16 bit patterns; each value is widened exactly to double.
+ *   - inputs are 16-bit bit patterns, all bf16 or all IEEE binary16 (fp16, the input type of
+ *     the FlashMLA-ETAP summary's H20 figures, "Planteamiento del Problema"); each value is
+ *     widened exactly to double.
  *
  * Layouts (row-major, contiguous): q [B,Hq,Lq,d], k [B,Hkv,Lk,d], v [B,Hkv,Lk,ldv] with
  * the first dv columns used; outputs are double.
@@ -50,12 +52,41 @@
 #define ORACLE_MUTANT 0
 #endif
 
-/* bf16 bit pattern -> double, exact. */
-static double widen(uint16_t h) {
+enum { ELEM_BF16 = 0, ELEM_F16 = 1 };
+
+/* bf16 bit pattern -> double, exact (bf16 is the upper half of an IEEE binary32). */
+static double widen_bf16(uint16_t h) {
     uint32_t u = ((uint32_t)h) << 16;
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/*
+ * IEEE 754 binary16 bit pattern -> double, exact, from the format's definition: sign bit 15,
+ * 5-bit biased exponent e (bias 15) in bits 10-14, 10-bit fraction f. e = 0 is zero or
+ * subnormal, f * 2^-24; 1 <= e <= 30 is (1024 + f) * 2^(e - 25); e = 31 is +-inf (f = 0)
+ * or NaN. Every binary16 value is a double, so ldexp is exact.
+ */
+static double widen_f16(uint16_t h) {
+    int s = h >> 15, e = (h >> 10) & 31, f = h & 1023;
+    double mag;
+    if (e == 31) {
+        mag = f == 0 ? INFINITY : NAN;
+    } else if (e == 0) {
+#if ORACLE_MUTANT == 9
+        mag = ldexp((double)(1024 + f), -24); /* planted: implicit leading one on subnormals */
+#else
+        mag = ldexp((double)f, -24);
+#endif
+    } else {
+        mag = ldexp((double)(1024 + f), e - 25);
+    }
+    return s ? -mag : mag;
+}
+
+static double widen(int elem, uint16_t h) {
+    return elem == ELEM_F16 ? widen_f16(h) : widen_bf16(h);
 }
 
 typedef struct {
@@ -64,6 +95,7 @@ typedef struct {
     double scale;
     int causal;
     int64_t kv_begin, kv_end;
+    int elem;
 } problem;
 
 static int check_problem(const problem *p) {
@@ -72,6 +104,7 @@ static int check_problem(const problem *p) {
     if (p->d < 1 || p->dv < 1 || p->ldv < p->dv) return 1;
     if (p->Hq % p->Hkv != 0) return 1;
     if (p->kv_begin < 0 || p->kv_end > p->Lk || p->kv_begin > p->kv_end) return 1;
+    if (p->elem != ELEM_BF16 && p->elem != ELEM_F16) return 1;
     return 0;
 }
 
@@ -102,12 +135,12 @@ static double dot_qk(const problem *p, int64_t b, int64_t h, int64_t i, int64_t 
     double a0 = 0, a1 = 0, a2 = 0, a3 = 0;
     int64_t c = 0;
     for (; c + 4 <= p->d; c += 4) {
-        a0 += widen(qr[c + 0]) * widen(kr[c + 0]);
-        a1 += widen(qr[c + 1]) * widen(kr[c + 1]);
-        a2 += widen(qr[c + 2]) * widen(kr[c + 2]);
-        a3 += widen(qr[c + 3]) * widen(kr[c + 3]);
+        a0 += widen(p->elem, qr[c + 0]) * widen(p->elem, kr[c + 0]);
+        a1 += widen(p->elem, qr[c + 1]) * widen(p->elem, kr[c + 1]);
+        a2 += widen(p->elem, qr[c + 2]) * widen(p->elem, kr[c + 2]);
+        a3 += widen(p->elem, qr[c + 3]) * widen(p->elem, kr[c + 3]);
     }
-    for (; c < p->d; ++c) a0 += widen(qr[c]) * widen(kr[c]);
+    for (; c < p->d; ++c) a0 += widen(p->elem, qr[c]) * widen(p->elem, kr[c]);
     return (a0 + a1) + (a2 + a3);
 }
 
@@ -116,9 +149,9 @@ static double v_at(const problem *p, int64_t b, int64_t hkv, int64_t j, int64_t 
     /* planted: operand indexed transposed (column-major read of a row-major V) */
     int64_t flat = c * p->Lk + j;
     int64_t jj = flat / p->ldv % p->Lk, cc = flat % p->ldv;
-    return widen(p->v[((b * p->Hkv + hkv) * p->Lk + jj) * p->ldv + cc]);
+    return widen(p->elem, p->v[((b * p->Hkv + hkv) * p->Lk + jj) * p->ldv + cc]);
 #else
-    return widen(p->v[((b * p->Hkv + hkv) * p->Lk + j) * p->ldv + c]);
+    return widen(p->elem, p->v[((b * p->Hkv + hkv) * p->Lk + j) * p->ldv + c]);
 #endif
 }
 
@@ -213,9 +246,9 @@ static void *run_job(void *arg) {
 int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
                      int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d, int64_t dv,
                      int64_t ldv, double scale, int causal, int64_t kv_begin, int64_t kv_end,
-                     const int64_t *rows, int64_t n_rows, double *o, double *lse,
+                     const int64_t *rows, int64_t n_rows, double *o, double *lse, int elem,
                      int nthreads) {
-    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, kv_begin, kv_end};
+    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, kv_begin, kv_end, elem};
     if (check_problem(&p) || (n_rows > 0 && (!rows || !o || !lse)) || n_rows < 0) return 1;
     int64_t total = B * Hq * Lq;
     for (int64_t r = 0; r < n_rows; ++r)
@@ -247,8 +280,8 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
 /* The probability row P[i, :] (length Lk, zero at masked keys) of one flat row id. */
 int oracle_softmax_row(const uint16_t *q, const uint16_t *k, int64_t B, int64_t Hq,
                        int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d, double scale,
-                       int causal, int64_t row, double *p_out) {
-    problem p = {q, k, k, B, Hq, Hkv, Lq, Lk, d, 1, d, scale, causal, 0, Lk};
+                       int causal, int64_t row, double *p_out, int elem) {
+    problem p = {q, k, k, B, Hq, Hkv, Lq, Lk, d, 1, d, scale, causal, 0, Lk, elem};
     if (check_problem(&p) || row < 0 || row >= B * Hq * Lq || !p_out) return 1;
     double *s = (double *)malloc((size_t)Lk * sizeof(double));
     double *pr = (double *)malloc((size_t)Lk * sizeof(double));
@@ -269,8 +302,8 @@ int oracle_softmax_row(const uint16_t *q, const uint16_t *k, int64_t B, int64_t 
 int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                 int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
                                 int64_t d, int64_t dv, int64_t ldv, double scale, int causal,
-                                int64_t b, int64_t h, double *o, double *lse) {
-    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, 0, Lk};
+                                int64_t b, int64_t h, double *o, double *lse, int elem) {
+    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, 0, Lk, elem};
     if (check_problem(&p) || b < 0 || b >= B || h < 0 || h >= Hq || !o || !lse) return 1;
     int64_t hkv = kv_head_of(&p, h);
     double *St = (double *)malloc((size_t)(Lk * Lq) * sizeof(double));
@@ -282,7 +315,7 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
         for (int64_t i = 0; i < Lq; ++i) {
             const uint16_t *qr = q + ((b * Hq + h) * Lq + i) * d;
             double acc = 0.0;
-            for (int64_t c = 0; c < d; ++c) acc += widen(kr[c]) * widen(qr[c]);
+            for (int64_t c = 0; c < d; ++c) acc += widen(elem, kr[c]) * widen(elem, qr[c]);
             St[j * Lq + i] = visible(&p, i, j) ? scale * acc : -INFINITY;
         }
     }
@@ -308,7 +341,7 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
         for (int64_t i = 0; i < Lq; ++i) {
             double acc = 0.0;
             for (int64_t j = 0; j < Lk; ++j)
-                acc += widen(v[((b * Hkv + hkv) * Lk + j) * ldv + c]) * St[j * Lq + i];
+                acc += widen(elem, v[((b * Hkv + hkv) * Lk + j) * ldv + c]) * St[j * Lq + i];
             Ot[c * Lq + i] = acc;
         }
     /* O = Ot^T */
@@ -350,6 +383,14 @@ int oracle_combine(const double *o_parts, const double *lse_parts, int64_t n_spl
             for (int64_t c = 0; c < dv; ++c) o[r * dv + c] += w * o_parts[(s * n_rows + r) * dv + c];
         }
     }
+    return 0;
+}
+
+/* The exact widening the oracle applies: out[i] = value of the 16-bit pattern in[i] read as
+ * elem (0 = bf16, 1 = fp16). Returns 1 for an unknown elem. */
+int oracle_widen(const uint16_t *in, int64_t n, int elem, double *out) {
+    if ((elem != ELEM_BF16 && elem != ELEM_F16) || n < 0 || (n > 0 && (!in || !out))) return 1;
+    for (int64_t i = 0; i < n; ++i) out[i] = widen(elem, in[i]);
     return 0;
 }
 

@@ -10,7 +10,10 @@ Sources of the facts:
   * shared K/V heads (GQA FAQ of "Activar Flash Attention con llama.cpp");
   * closed forms and invariants of softmax (rows sum to one, shift invariance, constant and
     one-hot value rows, log-sum-exp merge of disjoint key sets);
-  * a library routine: torch's fp64 CPU scaled_dot_product_attention with an explicit mask;
+  * a library routine: torch's fp64 CPU scaled_dot_product_attention with an explicit mask,
+    for bf16 and for fp16 inputs;
+  * library conversions of every 16-bit pattern (numpy float16, torch bfloat16) for the
+    oracle's exact widening;
   * a hand-derived worked example in tests/golden/.
 """
 from __future__ import annotations
@@ -245,6 +248,43 @@ def pin_golden_worked_example(mutant=0):
         assert np.max(np.abs(lse[0, 0] - lse_ref)) <= 1e-12, case["name"]
 
 
+def pin_widen_tables(mutant=0):
+    """Every one of the 65536 bit patterns widens to the value numpy (fp16) and torch (bf16)
+    give it: IEEE binary16 incl. subnormals, infinities and NaN; bf16 likewise."""
+    bits = np.arange(65536, dtype=np.uint16)
+    got = oracle.widen(bits, "f16", mutant=mutant)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    got = oracle.widen(bits, "bf16", mutant=mutant)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def pin_library_sdpa_f16(mutant=0):
+    """fp16 inputs (some subnormal values in V) against torch's fp64 scaled_dot_product_attention."""
+    for n, (B, Hq, Hkv, Lq, Lk, d, dv, causal) in enumerate(SHAPES):
+        g = torch.Generator().manual_seed(150 + n)
+        q = torch.randn((B, Hq, Lq, d), generator=g).to(torch.float16)
+        k = torch.randn((B, Hkv, Lk, d), generator=g).to(torch.float16)
+        v = (torch.randn((B, Hkv, Lk, dv), generator=g) * 1e-5).to(torch.float16)
+        assert (v.abs() < 2.0 ** -14).any()  # subnormal fp16 values take part
+        o, lse = oracle.attn(q, k, v, mutant=mutant, **_args(B, Hq, Hkv, Lq, Lk, d, dv, causal))
+        G = Hq // Hkv
+        kr, vr = f64(k).repeat_interleave(G, 1), f64(v).repeat_interleave(G, 1)
+        mask = bottom_right_mask(Lq, Lk, causal)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            f64(q), kr, vr, attn_mask=mask, scale=1.0 / math.sqrt(d))
+        assert np.max(np.abs(o - ref.numpy())) <= 1e-12 * 1e-5
+        s = torch.einsum("bhid,bhjd->bhij", f64(q), kr) / math.sqrt(d)
+        ref_l = torch.logsumexp(s.masked_fill(~mask, -math.inf), dim=-1)
+        assert np.max(np.abs(lse - ref_l.numpy())) <= 1e-12
+
+
 ALL_PINS = [pin_rows_sum_to_one, pin_transposed_flow, pin_constant_v, pin_one_hot,
             pin_closed_forms, pin_shift_invariance, pin_gqa_equals_repeated_mha,
-            pin_split_merge, pin_library_sdpa, pin_latent_kv, pin_golden_worked_example]
+            pin_split_merge, pin_library_sdpa, pin_latent_kv, pin_golden_worked_example,
+            pin_widen_tables, pin_library_sdpa_f16]

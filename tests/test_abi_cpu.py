@@ -37,6 +37,9 @@ def lib():
     L.attn_decode_ex.argtypes = [vp] * 5 + [i] * 8 + [f, i, i, vp, sz, i, vp]
     L.attn_decode.argtypes = [vp] * 5 + [i] * 8 + [f, i, i, vp, sz, vp]
     L.attn_combine.argtypes = [vp] * 4 + [i] * 5 + [vp]
+    L.attn_fwd_typed.argtypes = [vp] * 5 + [i] * 7 + [f, i, i, vp]
+    L.attn_decode_typed.argtypes = [vp] * 5 + [i] * 8 + [f, i, i, vp, sz, i, i, vp]
+    L.attn_combine_typed.argtypes = [vp] * 4 + [i] * 6 + [vp]
     L.attn_decode_workspace_size.argtypes = [i] * 7
     L.attn_decode_workspace_size.restype = sz
     L.attn_status_string.argtypes = [i]
@@ -65,7 +68,7 @@ def test_status_strings(lib):
         seen.add(s)
     assert len(seen) == 7
     assert lib.attn_status_string(99).decode() == "unknown status"
-    assert lib.attn_abi_version() == 10000
+    assert lib.attn_abi_version() == 10100
 
 
 def fwd(lib, q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128, scale=0.1,
@@ -149,3 +152,42 @@ def test_binding_has_c_names():
     for name in ("attn_fwd", "attn_decode", "attn_combine", "attn_decode_workspace_size", "attn_status_string",
                  "attn_check_device"):
         assert callable(getattr(attn, name))
+
+
+BF16, F16 = 0, 1
+
+
+@pytest.mark.parametrize("dtype", [BF16, F16])
+def test_typed_entry_points_check_like_untyped(lib, dtype):
+    """The *_typed entry points apply the same host checks for both element types."""
+    def fwd_t(**kw):
+        a = dict(q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128,
+                 scale=0.1, causal=1)
+        a.update(kw)
+        return lib.attn_fwd_typed(*a.values(), dtype, None)
+
+    def dec_t(**kw):
+        a = dict(q=A, k=B_, v=B_, o=D_, lse=None, B=2, Hq=16, Hkv=1, Lq=2, Lk=1000, d=576, dv=512,
+                 ldv=576, scale=0.04, causal=1, splits=4, ws=0x100000, ws_bytes=1 << 30, impl=0)
+        a.update(kw)
+        return lib.attn_decode_typed(*a.values(), dtype, None)
+
+    assert fwd_t(q=None) == INVALID
+    assert fwd_t(Hq=3, Hkv=2) == INVALID
+    assert fwd_t(d=96, dv=96) == UNSUPPORTED
+    assert fwd_t(q=A + 8) == MISALIGNED
+    assert dec_t(ldv=256) == INVALID
+    assert dec_t(Hq=64) == UNSUPPORTED
+    assert dec_t(ws=None) == WORKSPACE
+    assert dec_t(k=B_ + 4, v=B_ + 4) == MISALIGNED
+    assert lib.attn_combine_typed(A, B_, C_, None, 1, 2, 3, 62, 4, dtype, None) == MISALIGNED
+    assert lib.attn_combine_typed(None, B_, C_, None, 1, 2, 3, 64, 4, dtype, None) == INVALID
+
+
+@pytest.mark.parametrize("bad", [-1, 2, 7])
+def test_typed_entry_points_reject_unknown_dtype(lib, bad):
+    # arguments otherwise valid: only the element type is wrong, so nothing reaches a launch
+    assert lib.attn_fwd_typed(A, B_, C_, D_, None, 1, 2, 1, 128, 128, 128, 128, 0.1, 1, bad, None) == INVALID
+    assert lib.attn_decode_typed(A, B_, B_, D_, None, 2, 16, 1, 2, 1000, 576, 512, 576, 0.04, 1, 4,
+                                 0x100000, 1 << 30, 0, bad, None) == INVALID
+    assert lib.attn_combine_typed(A, B_, C_, None, 1, 2, 3, 64, 4, bad, None) == INVALID
