@@ -340,8 +340,12 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   p.G = Hq / Hkv;
   p.n_pairs = (n_qtiles + 1) / 2;
   const long long units = (long long)p.n_pairs * B * Hq;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (units > 0x7fff0000LL) return ATTN_ERR_UNSUPPORTED;  // room for one more round of unit ids
   p.n_units = (int)units;
+  // scheduling groups of batches whose K/V (Hkv * Lk rows of d + dv elements each) stays within
+  // 64 MiB, about half of the L2
+  const long long kv_per_batch = (long long)Hkv * Lk * (d + d) * 2;
+  p.group_b = (int)std::max(1LL, std::min<long long>(B, (64LL << 20) / std::max(1LL, kv_per_batch)));
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   // persistent grid: one CTA per SM (fewer when there are fewer work units)

@@ -35,15 +35,17 @@ struct Prefill2Params {
   int B, Hq, Hkv, Lq, Lk, G;
   int n_pairs;  // ceil(ceil(Lq / 128) / 2)
   int n_units;  // n_pairs * B * Hq
+  int group_b;  // batches per scheduling group (their K/V fits comfortably in L2)
   int causal;
   float scale_log2;
 };
 
 #ifndef ATTN_EXP2_EMULATE_MASK
-#define ATTN_EXP2_EMULATE_MASK 0x8888u
+#define ATTN_EXP2_EMULATE_MASK 0x8080u
 #endif
 // Key pairs e (0..15 within each group of 32 keys) whose exponentials are computed with the FMA
-// polynomial (bit e set) instead of ex2.approx on the MUFU unit.
+// polynomial (bit e set) instead of ex2.approx on the MUFU unit. One pair in eight measured best
+// on B200 (8K causal prefill: none 1116, 1/8 1135, 1/4 1099, 3/8 1093, 1/2 1071 TFLOP/s).
 constexpr uint32_t kExp2EmulateMask = ATTN_EXP2_EMULATE_MASK;
 
 template <int D>
@@ -52,11 +54,12 @@ struct Prefill2Cfg {
   static constexpr int DC = D / 64;
   static constexpr int CHUNK = 128 * 128;
   static constexpr int Q_BYTES = DC * CHUNK;
-  static constexpr int KV_BYTES = DC * CHUNK;
-  static constexpr int NS = (D == 128) ? 4 : 6;
+  static constexpr int KV_BYTES = DC * CHUNK;       // one K or V tile
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;  // ring stage j holds (K_j, V_j)
+  static constexpr int NS = (D == 128) ? 2 : 3;
   static constexpr int OFF_Q = 0;  // Q_A, then Q_B
   static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * STAGE_BYTES;
   // q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], o_free[2], drain
   static constexpr int N_BARS = 2 + 2 * NS + 8 + 1;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
@@ -83,19 +86,34 @@ struct UnitCoords {
   int b, h, q0;
 };
 
-// Unit order: batch-major, then heaviest (last) query-tile pairs first, then heads. CTAs take
-// units round-robin, so the units in flight at any time belong to one or two batches and share
-// their K/V in L2 (ordering heaviest-first across all batches made every batch's K/V live at once
-// and doubled the DRAM reads of a 16-batch prefill); within a batch the light causal pairs come
-// last, which keeps the tail short.
+// Unit order. Batches are taken in groups of group_b whose K/V together fits in L2 with room to
+// spare; within a group the units are sorted by cost (heaviest query-tile pair first: under a
+// causal mask the cost of a pair grows with its position), then by batch, then by head, so that
+// sibling query heads of a kv head are adjacent and share their K/V tiles in L2. (Taking the
+// heaviest pairs of all batches first would keep every batch's K/V live at once and, for a
+// 16-batch 2K prefill, doubled the DRAM reads.)
 __device__ __forceinline__ UnitCoords prefill_unit(const Prefill2Params& p, int u) {
   const int per_batch = p.n_pairs * p.Hq;
-  const int rem = u % per_batch;
+  const int per_group = p.group_b * per_batch;
+  const int g = u / per_group;
+  const int b0 = g * p.group_b;
+  const int gb = min(p.group_b, p.B - b0);
+  const int w = u - g * per_group;
+  const int lvl = w / (gb * p.Hq);
+  const int rem = w - lvl * gb * p.Hq;
   UnitCoords c;
-  c.b = u / per_batch;
-  c.h = rem % p.Hq;  // sibling query heads of a kv head are adjacent
-  c.q0 = (p.n_pairs - 1 - rem / p.Hq) * 256;
+  c.b = b0 + rem / p.Hq;
+  c.h = rem % p.Hq;
+  c.q0 = (p.n_pairs - 1 - lvl) * 256;
   return c;
+}
+
+// The k-th unit of CTA `cta` among `grid` persistent CTAs: units are dealt in rounds of `grid`,
+// in CTA order on even rounds and in reverse order on odd rounds. On the cost-sorted sequence
+// this evens out the per-CTA totals (plain round-robin gives CTA 0 the heaviest unit of every
+// round: 12 % longer critical path on an 8K causal prefill).
+__device__ __forceinline__ int prefill_unit_index(int k, int cta, int grid) {
+  return k * grid + ((k & 1) ? grid - 1 - cta : cta);
 }
 
 template <int D, typename E>
@@ -153,18 +171,22 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       tma_prefetch_desc(&tm_v);
       bool ok = true;
       int kv_t = 0, qc = 0;
-      auto load_kv = [&](const CUtensorMap* m, int tile, int zkv) {
+      // stage kv_t % NS receives K and V of one key tile under a single full barrier
+      auto load_kv = [&](int tile, int zkv) {
         const int s = kv_t % C::NS;
         if (kv_t >= C::NS) ok = mbar_wait(bar_kv_empty + 8 * s, ((kv_t / C::NS) & 1) ^ 1, 61);
         if (!ok) return;
         const uint32_t full = bar_kv_full + 8 * s;
-        mbar_arrive_expect_tx(full, C::KV_BYTES);
+        const uint32_t dst = base + C::OFF_KV + s * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(full, C::STAGE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::DC; ++c) tma_load_3d(dst + c * C::CHUNK, &tm_k, full, 64 * c, tile * C::BN, zkv);
 #pragma unroll
         for (int c = 0; c < C::DC; ++c)
-          tma_load_3d(base + C::OFF_KV + s * C::KV_BYTES + c * C::CHUNK, m, full, 64 * c, tile * C::BN, zkv);
+          tma_load_3d(dst + C::KV_BYTES + c * C::CHUNK, &tm_v, full, 64 * c, tile * C::BN, zkv);
         ++kv_t;
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
         const UnitCoords uc = prefill_unit(p, u);
         const int nA = prefill_kv_tiles(p, uc.q0), nB = prefill_kv_tiles(p, uc.q0 + 128);
         const int n = max(nA, nB);
@@ -180,10 +202,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
         }
         ++qc;
-        for (int j = 0; j < n && ok; ++j) {
-          load_kv(&tm_k, j, zkv);
-          if (ok) load_kv(&tm_v, j, zkv);
-        }
+        for (int j = 0; j < n && ok; ++j) load_kv(j, zkv);
       }
       if (!ok) {
         if (qc > 0) mbar_wait_drain(bar_q_full, (qc - 1) & 1);
@@ -202,8 +221,8 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         ok = mbar_wait(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site);
         if (ok) tc_fence_after();
       };
-      auto issue_s = [&](int x, int kidx) {
-        const uint32_t kb = base + C::OFF_KV + (kidx % C::NS) * C::KV_BYTES;
+      auto issue_s = [&](int x, int sidx) {
+        const uint32_t kb = base + C::OFF_KV + (sidx % C::NS) * C::STAGE_BYTES;
         const uint32_t qb = base + C::OFF_Q + x * C::Q_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -214,7 +233,11 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         mma_commit(bar_s_full + 8 * x);
         issued = true;
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      // Per key tile j the only wait between the last S product of tile j and the first P.V
+      // product of tile j+1 is the one on P: the stage of tile j is released right after its
+      // last P.V product (one commit, while the tensor core still has S work queued), and the
+      // stage of tile j+1 is awaited before the first S of tile j+1.
+      for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
         const UnitCoords uc = prefill_unit(p, u);
         int nX[2];
         nX[0] = prefill_kv_tiles(p, uc.q0);
@@ -224,17 +247,15 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         if (!ok) break;
         ++qc;
         tc_fence_after();
-        wait_stage(kv_t, 64);  // K_0
+        wait_stage(kv_t, 64);  // K_0, V_0
         if (!ok) break;
         for (int x = 0; x < 2; ++x)
           if (nX[x] > 0) issue_s(x, kv_t);
-        mma_commit(bar_kv_empty + 8 * (kv_t % C::NS));
         if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
         for (int j = 0; j < n && ok; ++j) {
-          const int vi = kv_t + 2 * j + 1, ki = kv_t + 2 * j + 2;
-          wait_stage(vi, 65);  // V_j
-          if (!ok) break;
-          bool k_next = false;
+          const int si = kv_t + j;                // stage of tile j
+          const int x_last = (j < nX[1]) ? 1 : 0;  // last tile whose P.V reads V_j
+          bool next_ready = false;
           for (int x = 0; x < 2 && ok; ++x) {
             if (j >= nX[x]) continue;
             if (j == 0 && units_done[x] > 0) {
@@ -245,20 +266,22 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             if (!ok) break;
             ++p_cnt[x];
             tc_fence_after();
-            const uint32_t vb = base + C::OFF_KV + (vi % C::NS) * C::KV_BYTES;
+            const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
 #pragma unroll
             for (int kk = 0; kk < C::BN / 16; ++kk) {
               const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
               // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
               mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
             }
+            // K_j was last read by S of tile j (issued earlier), V_j by this product
+            if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
             if (j + 1 < nX[x]) {
-              if (!k_next) {
-                wait_stage(ki, 68);  // K_{j+1}
+              if (!next_ready) {
+                wait_stage(si + 1, 68);  // K_{j+1}, V_{j+1}
                 if (!ok) break;
-                k_next = true;
+                next_ready = true;
               }
-              issue_s(x, ki);
+              issue_s(x, si + 1);
             }
             if (j == nX[x] - 1) {
               mma_commit(bar_o_ready + 8 * x);
@@ -266,13 +289,11 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             }
           }
           if (!ok) break;
-          mma_commit(bar_kv_empty + 8 * (vi % C::NS));
-          if (k_next) mma_commit(bar_kv_empty + 8 * (ki % C::NS));
           // Q may be reloaded once the last S of this unit (issued in iteration n-2) is done
           if (j == n - 2) mma_commit(bar_q_empty);
         }
         if (!ok) break;
-        kv_t += 2 * n;
+        kv_t += n;
       }
       if (!ok && issued) {
         mma_commit(bar_drain);
@@ -289,7 +310,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     const int off = p.Lk - p.Lq;
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
       const UnitCoords uc = prefill_unit(p, u);
       const int qx0 = uc.q0 + 128 * x;
       const int nt = prefill_kv_tiles(p, qx0);
