@@ -130,7 +130,8 @@ int split_chunk(int Lk, int splits) {
 // fixed start-up/drain cost of about kFixedTiles tiles (barrier set-up, Q load, ring fill, partial
 // write), and every split adds partial-result traffic. Minimise
 //   waves * (tiles per split + kFixedTiles) * (1 + partial bytes / KV bytes).
-// (On B200: mla_decode_64k -> 9 splits, gqa_decode_32k -> 8, both the measured best.)
+// (On B200: mla_decode_64k -> 9 splits at one CTA per SM, gqa_decode_32k -> 9 at two CTAs per
+// SM, both the measured best: 4 to 28 splits were timed.)
 int choose_splits(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int sms, int ctas_per_sm) {
   constexpr double kFixedTiles = 5.0, kTileKeys = 48.0;
   const long long units = (long long)B * Hkv;
@@ -153,6 +154,22 @@ int choose_splits(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int sms, int c
     }
   }
   return best;
+}
+
+// CTAs per SM of the dense-V (d = 128) queries-on-M decode kernel: bounded by shared memory
+// (228 KB per SM, 1 KB reserved per CTA) and by TMEM (512 columns, 256 per CTA).
+using DenseTn128Cfg = attn::DecodeTnCfg<2, 1, 48, 3, true>;
+constexpr int kDenseTn128Occupancy = 233472 / (DenseTn128Cfg::SMEM_BYTES + 1024);
+static_assert(kDenseTn128Occupancy == 2, "dense-V decode sized for two CTAs per SM");
+
+// Which kernel attn_decode runs for impl == ATTN_DECODE_AUTO.
+int auto_impl(const void* k, const void* v, int Hq, int Hkv, int Lq, int d, int dv, int ldv) {
+  return tn_supported(k, v, Hq, Hkv, Lq, d, dv, ldv) ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
+}
+
+// CTAs per SM the split model assumes for a (resolved) kernel choice.
+int decode_ctas_per_sm(int impl, bool dense_v, int d) {
+  return (impl == ATTN_DECODE_TCGEN05_N && dense_v && d == 128) ? kDenseTn128Occupancy : 1;
 }
 
 template <int RMAX, int CPT, typename E>
@@ -205,19 +222,19 @@ attn_status launch_tc_nb(const DecodeParams& p, int splits, cudaStream_t st) {
 // Key tile and stage count of the queries-on-M decode kernel (chosen by measurement on B200).
 constexpr int kTnBK = ATTN_TN_BK, kTnNST = ATTN_TN_NST;
 
-template <int DCH, int NPIECE, int NST, bool SEPV, typename E>
+template <int DCH, int NPIECE, int NST, bool SEPV, typename E, int BK = kTnBK>
 attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
-  using C = attn::DecodeTnCfg<DCH, NPIECE, kTnBK, NST, SEPV>;
+  using C = attn::DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>;
   CUtensorMap tq, tkv, tv;
   if (!encode16<E>(&tq, p.q, (uint64_t)p.d, (uint64_t)p.rows_total, 0, 64, 32)) return ATTN_ERR_CUDA;
-  if (!encode16<E>(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK)) return ATTN_ERR_CUDA;
+  if (!encode16<E>(&tkv, p.k, (uint64_t)p.d, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, BK)) return ATTN_ERR_CUDA;
   if (SEPV) {
-    if (!encode16<E>(&tv, p.v, (uint64_t)p.dv, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, kTnBK, (uint64_t)p.ldv))
+    if (!encode16<E>(&tv, p.v, (uint64_t)p.dv, (uint64_t)p.Lk, (uint64_t)p.B * p.Hkv, 64, BK, (uint64_t)p.ldv))
       return ATTN_ERR_CUDA;
   } else {
     tv = tkv;  // unused
   }
-  auto kern = attn::decode_tn_kernel<DCH, NPIECE, kTnBK, NST, SEPV, E>;
+  auto kern = attn::decode_tn_kernel<DCH, NPIECE, BK, NST, SEPV, E>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, tv, p);
@@ -233,8 +250,9 @@ attn_status launch_tn_np(const DecodeParams& p, int splits, cudaStream_t st) {
 template <typename E>
 attn_status launch_tn_any(const DecodeParams& p, int splits, cudaStream_t st) {
   if (!p.v_is_k) {
-    // dense V beside K in each stage (small stages: a deeper ring)
-    if (p.d == 128) return launch_tn<2, 1, 6, true, E>(p, splits, st);
+    // dense V beside K in each stage; d = 128: a 3-stage ring small enough for two CTAs per SM
+    // (each CTA's start-up, drain and per-tile waits hide behind the other's streaming)
+    if (p.d == 128) return launch_tn<2, 1, 3, true, E, 48>(p, splits, st);
     if (p.d == 256) return launch_tn<4, 1, 3, true, E>(p, splits, st);
     return ATTN_ERR_UNSUPPORTED;
   }
@@ -375,12 +393,14 @@ attn_status decode_impl(const void* q, const void* k, const void* v, void* o, fl
   const bool tc_ok = tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
   const bool tn_ok = tn_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
   const bool cc_ok = cc_supported(Hq, Hkv, Lq, d, dv, ldv);
-  if (impl == ATTN_DECODE_AUTO) impl = tn_ok ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
+  if (impl == ATTN_DECODE_AUTO) impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
   if (impl == ATTN_DECODE_TCGEN05_T && !tc_ok) return ATTN_ERR_UNSUPPORTED;
   if (impl == ATTN_DECODE_TCGEN05_N && !tn_ok) return ATTN_ERR_UNSUPPORTED;
   if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
+  const bool dense_v = !(v == k && ldv == d);
   int splits = num_splits;
-  if (splits == 0) splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  if (splits == 0)
+    splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), decode_ctas_per_sm(impl, dense_v, d));
   const long long rows = (long long)B * Hq * Lq;
   const size_t need = workspace_bytes(rows, dv, splits);
   if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
@@ -460,14 +480,20 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv, int num_splits) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || dv < 1 || num_splits < 0 || num_splits > 256) return 0;
   if (Hq % Hkv != 0) return 0;
-  int s = num_splits;
-  if (s == 0) s = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
-  return workspace_bytes((long long)B * Hq * Lq, dv, s);
+  if (num_splits > 0) return workspace_bytes((long long)B * Hq * Lq, dv, num_splits);
+  // enough for the count attn_decode chooses with either kernel occupancy
+  const int sms = current_sm_count();
+  const int s1 = choose_splits(B, Hq, Hkv, Lq, Lk, dv, sms, 1);
+  const int s2 = choose_splits(B, Hq, Hkv, Lq, Lk, dv, sms, kDenseTn128Occupancy);
+  return workspace_bytes((long long)B * Hq * Lq, dv, std::max(s1, s2));
 }
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
-  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  // dv == d == 128 is taken to be a dense V on the queries-on-M kernel (the GQA decode shape)
+  const int R = (Hq / Hkv) * Lq;
+  const int occ = (dv == d && d == 128 && R <= 32) ? kDenseTn128Occupancy : 1;
+  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), occ);
 }
 
 attn_status attn_decode_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -534,7 +560,11 @@ attn_status attn_decode_noalloc(const void* q, const void* k, const void* v, voi
   attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
   if (st != ATTN_OK) return st;
   if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
-  const int splits = num_splits > 0 ? num_splits : choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), 1);
+  const int impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
+  const int splits =
+      num_splits > 0 ? num_splits
+                     : choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(),
+                                     decode_ctas_per_sm(impl, !(v == k && ldv == d), d));
   const size_t need = workspace_bytes((long long)B * Hq * Lq, dv, splits);
   if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -191,3 +191,14 @@ def test_typed_entry_points_reject_unknown_dtype(lib, bad):
     assert lib.attn_decode_typed(A, B_, B_, D_, None, 2, 16, 1, 2, 1000, 576, 512, 576, 0.04, 1, 4,
                                  0x100000, 1 << 30, 0, bad, None) == INVALID
     assert lib.attn_combine_typed(A, B_, C_, None, 1, 2, 3, 64, 4, bad, None) == INVALID
+
+
+def test_default_workspace_covers_default_splits(lib):
+    """num_splits = 0 sizes the workspace for whichever split count attn_decode will choose."""
+    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 7
+    for B, Hq, Hkv, Lq, Lk, d, dv in [(16, 32, 8, 1, 32768, 128, 128), (32, 16, 1, 2, 65536, 576, 512),
+                                      (2, 8, 2, 1, 777, 128, 128), (4, 16, 2, 2, 5000, 256, 256)]:
+        s = lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv)
+        assert 1 <= s <= 256
+        assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, 0) >= \
+            lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, s)
