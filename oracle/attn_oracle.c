@@ -35,8 +35,16 @@
  *     the FlashMLA-ETAP summary's H20 figures, "Planteamiento del Problema"); each value is
  *     widened exactly to double.
  *
+ *   MInference article (7minutos.es), on the sparse patterns of long-context prefill (A-shape,
+ *   vertical bar, block-sparse): with a given sparse index the attention stays the exact
+ *   softmax, restricted to the listed keys. Reading taken for the block form: query rows are
+ *   cut into blocks of blk_q rows and keys into blocks of blk_k keys; query block qb of head
+ *   (b, h) sees exactly the key blocks in its list (and the causal mask still applies). A row
+ *   that sees no key gets O = 0 and LSE = -inf.
+ *
  * Layouts (row-major, contiguous): q [B,Hq,Lq,d], k [B,Hkv,Lk,d], v [B,Hkv,Lk,ldv] with
- * the first dv columns used; outputs are double.
+ * the first dv columns used; outputs are double. Block lists: cnt [B,Hq,ceil(Lq/blk_q)] and
+ * idx [B,Hq,ceil(Lq/blk_q),max_blk] (int32; the first cnt entries of each list are used).
  *
  * Build: gcc -O2 -shared -fPIC -pthread attn_oracle.c -o liboracle.so -lm
  * ORACLE_MUTANT (compile-time, default 0) plants one deliberate mistake; only the mutation
@@ -96,6 +104,8 @@ typedef struct {
     int causal;
     int64_t kv_begin, kv_end;
     int elem;
+    const int32_t *blk_idx, *blk_cnt; /* NULL: dense */
+    int64_t max_blk, blk_q, blk_k;
 } problem;
 
 static int check_problem(const problem *p) {
@@ -105,6 +115,17 @@ static int check_problem(const problem *p) {
     if (p->Hq % p->Hkv != 0) return 1;
     if (p->kv_begin < 0 || p->kv_end > p->Lk || p->kv_begin > p->kv_end) return 1;
     if (p->elem != ELEM_BF16 && p->elem != ELEM_F16) return 1;
+    if (p->blk_cnt) {
+        if (!p->blk_idx || p->blk_q < 1 || p->blk_k < 1 || p->max_blk < 0) return 1;
+        const int64_t nqb = (p->Lq + p->blk_q - 1) / p->blk_q, nkb = (p->Lk + p->blk_k - 1) / p->blk_k;
+        for (int64_t s = 0; s < p->B * p->Hq * nqb; ++s) {
+            if (p->blk_cnt[s] < 0 || p->blk_cnt[s] > p->max_blk) return 1;
+            for (int32_t t = 0; t < p->blk_cnt[s]; ++t) {
+                const int32_t kb = p->blk_idx[s * p->max_blk + t];
+                if (kb < 0 || kb >= nkb) return 1;
+            }
+        }
+    }
     return 0;
 }
 
@@ -117,9 +138,27 @@ static int64_t kv_head_of(const problem *p, int64_t h) {
 #endif
 }
 
-/* Is key j visible to query row i? */
-static int visible(const problem *p, int64_t i, int64_t j) {
+/* Is key j in one of the key blocks listed for the query block of row i of head (b, h)? */
+static int listed(const problem *p, int64_t b, int64_t h, int64_t i, int64_t j) {
+    if (!p->blk_cnt) return 1;
+    const int64_t nqb = (p->Lq + p->blk_q - 1) / p->blk_q;
+    const int64_t slot = (b * p->Hq + h) * nqb + i / p->blk_q;
+    const int64_t kb = j / p->blk_k;
+    const int32_t *lst = p->blk_idx + slot * p->max_blk;
+    for (int32_t t = 0; t < p->blk_cnt[slot]; ++t) {
+#if ORACLE_MUTANT == 10
+        if (kb <= lst[t]) return 1; /* planted: the list read as an upper bound */
+#else
+        if (lst[t] == kb) return 1;
+#endif
+    }
+    return 0;
+}
+
+/* Is key j visible to query row i of head (b, h)? */
+static int visible(const problem *p, int64_t b, int64_t h, int64_t i, int64_t j) {
     if (j < p->kv_begin || j >= p->kv_end) return 0;
+    if (!listed(p, b, h, i, j)) return 0;
     if (!p->causal) return 1;
 #if ORACLE_MUTANT == 4
     return j <= i; /* planted: top-left alignment */
@@ -172,7 +211,7 @@ static void one_row(const problem *p, int64_t row, double *s, double *pr, double
     double m = -INFINITY;
     int64_t n_vis = 0;
     for (int64_t j = 0; j < p->Lk; ++j) {
-        if (!visible(p, i, j)) { s[j] = -INFINITY; continue; }
+        if (!visible(p, b, h, i, j)) { s[j] = -INFINITY; continue; }
 #if ORACLE_MUTANT == 7
         s[j] = dot_qk(p, b, h, i, j); /* planted: scale dropped */
 #else
@@ -243,14 +282,11 @@ static void *run_job(void *arg) {
  * split partial: O normalised by its own sum and the LSE of that range.
  * o: n_rows x dv, lse: n_rows. Returns 0 on success, 1 on bad arguments, 2 on no memory.
  */
-int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
-                     int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d, int64_t dv,
-                     int64_t ldv, double scale, int causal, int64_t kv_begin, int64_t kv_end,
-                     const int64_t *rows, int64_t n_rows, double *o, double *lse, int elem,
-                     int nthreads) {
-    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, kv_begin, kv_end, elem};
+static int run_rows(const problem *pp, const int64_t *rows, int64_t n_rows, double *o, double *lse,
+                    int nthreads) {
+    problem p = *pp;
     if (check_problem(&p) || (n_rows > 0 && (!rows || !o || !lse)) || n_rows < 0) return 1;
-    int64_t total = B * Hq * Lq;
+    int64_t total = p.B * p.Hq * p.Lq;
     for (int64_t r = 0; r < n_rows; ++r)
         if (rows[r] < 0 || rows[r] >= total) return 1;
     if (nthreads < 1) nthreads = 1;
@@ -277,11 +313,44 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
     return err;
 }
 
+/*
+ * Attention for a list of query rows. rows[r] is the flat row id (b*Hq + h)*Lq + i.
+ * Only keys in [kv_begin, kv_end) take part (the whole row: 0, Lk); a sub-range gives the
+ * split partial: O normalised by its own sum and the LSE of that range.
+ * o: n_rows x dv, lse: n_rows. Returns 0 on success, 1 on bad arguments, 2 on no memory.
+ */
+int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                     int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d, int64_t dv,
+                     int64_t ldv, double scale, int causal, int64_t kv_begin, int64_t kv_end,
+                     const int64_t *rows, int64_t n_rows, double *o, double *lse, int elem,
+                     int nthreads) {
+    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, kv_begin, kv_end, elem,
+                 NULL, NULL, 0, 1, 1};
+    return run_rows(&p, rows, n_rows, o, lse, nthreads);
+}
+
+/*
+ * Block-sparse attention for a list of query rows: as oracle_attn_rows over all keys, with
+ * key j visible to row i of head (b, h) only if block j / blk_k is in the list of query block
+ * i / blk_q (lists: cnt [B,Hq,nqb], idx [B,Hq,nqb,max_blk], entries in [0, ceil(Lk/blk_k))).
+ */
+int oracle_attn_rows_sparse(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                            int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d,
+                            int64_t dv, int64_t ldv, double scale, int causal, int64_t blk_q,
+                            int64_t blk_k, const int32_t *blk_idx, const int32_t *blk_cnt,
+                            int64_t max_blk, const int64_t *rows, int64_t n_rows, double *o,
+                            double *lse, int elem, int nthreads) {
+    if (!blk_cnt) return 1;
+    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, 0, Lk, elem,
+                 blk_idx, blk_cnt, max_blk, blk_q, blk_k};
+    return run_rows(&p, rows, n_rows, o, lse, nthreads);
+}
+
 /* The probability row P[i, :] (length Lk, zero at masked keys) of one flat row id. */
 int oracle_softmax_row(const uint16_t *q, const uint16_t *k, int64_t B, int64_t Hq,
                        int64_t Hkv, int64_t Lq, int64_t Lk, int64_t d, double scale,
                        int causal, int64_t row, double *p_out, int elem) {
-    problem p = {q, k, k, B, Hq, Hkv, Lq, Lk, d, 1, d, scale, causal, 0, Lk, elem};
+    problem p = {q, k, k, B, Hq, Hkv, Lq, Lk, d, 1, d, scale, causal, 0, Lk, elem, NULL, NULL, 0, 1, 1};
     if (check_problem(&p) || row < 0 || row >= B * Hq * Lq || !p_out) return 1;
     double *s = (double *)malloc((size_t)Lk * sizeof(double));
     double *pr = (double *)malloc((size_t)Lk * sizeof(double));
@@ -303,7 +372,7 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
                                 int64_t B, int64_t Hq, int64_t Hkv, int64_t Lq, int64_t Lk,
                                 int64_t d, int64_t dv, int64_t ldv, double scale, int causal,
                                 int64_t b, int64_t h, double *o, double *lse, int elem) {
-    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, 0, Lk, elem};
+    problem p = {q, k, v, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, 0, Lk, elem, NULL, NULL, 0, 1, 1};
     if (check_problem(&p) || b < 0 || b >= B || h < 0 || h >= Hq || !o || !lse) return 1;
     int64_t hkv = kv_head_of(&p, h);
     double *St = (double *)malloc((size_t)(Lk * Lq) * sizeof(double));
@@ -316,7 +385,7 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
             const uint16_t *qr = q + ((b * Hq + h) * Lq + i) * d;
             double acc = 0.0;
             for (int64_t c = 0; c < d; ++c) acc += widen(elem, kr[c]) * widen(elem, qr[c]);
-            St[j * Lq + i] = visible(&p, i, j) ? scale * acc : -INFINITY;
+            St[j * Lq + i] = visible(&p, b, h, i, j) ? scale * acc : -INFINITY;
         }
     }
     /* Pt = softmax over j of each column i (in place) */

@@ -62,6 +62,10 @@ def _lib(mutant: int = 0) -> ctypes.CDLL:
         L.oracle_attn_transposed_head.restype = ctypes.c_int
         L.oracle_attn_transposed_head.argtypes = [_u16p, _u16p, _u16p] + [_i64] * 8 + [
             ctypes.c_double, ctypes.c_int, _i64, _i64, _dp, _dp, ctypes.c_int]
+        L.oracle_attn_rows_sparse.restype = ctypes.c_int
+        L.oracle_attn_rows_sparse.argtypes = [_u16p, _u16p, _u16p] + [_i64] * 8 + [
+            ctypes.c_double, ctypes.c_int, _i64, _i64, ctypes.c_void_p, ctypes.c_void_p, _i64,
+            ctypes.POINTER(_i64), _i64, _dp, _dp, ctypes.c_int, ctypes.c_int]
         L.oracle_widen.restype = ctypes.c_int
         L.oracle_widen.argtypes = [_u16p, _i64, ctypes.c_int, _dp]
         L.oracle_combine.restype = ctypes.c_int
@@ -137,12 +141,16 @@ def default_threads() -> int:
 
 
 def attn_rows(q, k, v, rows, *, B, Hq, Hkv, Lq, Lk, d, dv, ldv=None, scale, causal,
-              kv_range=None, nthreads=None, elem=None, mutant: int = 0):
+              kv_range=None, blocks=None, nthreads=None, elem=None, mutant: int = 0):
     """O (n_rows x dv) and LSE (n_rows) for the flat row ids ``rows`` = (b*Hq + h)*Lq + i.
 
     ``kv_range=(j0, j1)`` restricts the keys to [j0, j1): the split partial (O normalised by its
     own sum, LSE of that range, -inf when no key is visible). ``v`` may be the same array as
     ``k`` (latent KV: V is the first dv columns of each K row, ldv = d).
+
+    ``blocks=(idx, cnt, blk_q, blk_k)`` gives block-sparse attention: idx int32
+    [B, Hq, ceil(Lq/blk_q), max_blk] and cnt int32 [B, Hq, ceil(Lq/blk_q)]; query block qb of head
+    (b, h) sees only the key blocks idx[b, h, qb, :cnt[b, h, qb]] (and the causal mask).
     """
     qb, kb, vb, ec = _operands(q, k, v, elem)
     ldv = dv if ldv is None else ldv
@@ -152,22 +160,36 @@ def attn_rows(q, k, v, rows, *, B, Hq, Hkv, Lq, Lk, d, dv, ldv=None, scale, caus
     lse = np.empty(rows.size, dtype=np.float64)
     assert qb.size == B * Hq * Lq * d and kb.size == B * Hkv * Lk * d
     assert vb.size == B * Hkv * Lk * ldv
-    rc = _lib(mutant).oracle_attn_rows(
-        _ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d, dv, ldv, float(scale), int(causal),
-        j0, j1, rows.ctypes.data_as(ctypes.POINTER(_i64)), rows.size, _dptr(o), _dptr(lse), ec,
-        nthreads or default_threads())
+    if blocks is not None:
+        if kv_range is not None:
+            raise ValueError("kv_range and blocks are exclusive")
+        idx, cnt, blk_q, blk_k = blocks
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+        cnt = np.ascontiguousarray(np.asarray(cnt, dtype=np.int32))
+        nqb = -(-Lq // blk_q)
+        assert cnt.shape == (B, Hq, nqb) and idx.shape[:3] == (B, Hq, nqb) and idx.ndim == 4
+        rc = _lib(mutant).oracle_attn_rows_sparse(
+            _ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d, dv, ldv, float(scale), int(causal),
+            int(blk_q), int(blk_k), _ptr(idx), _ptr(cnt), idx.shape[3],
+            rows.ctypes.data_as(ctypes.POINTER(_i64)), rows.size, _dptr(o), _dptr(lse), ec,
+            nthreads or default_threads())
+    else:
+        rc = _lib(mutant).oracle_attn_rows(
+            _ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d, dv, ldv, float(scale), int(causal),
+            j0, j1, rows.ctypes.data_as(ctypes.POINTER(_i64)), rows.size, _dptr(o), _dptr(lse), ec,
+            nthreads or default_threads())
     if rc != 0:
         raise ValueError(f"oracle_attn_rows rejected its arguments (code {rc})")
     return o, lse
 
 
 def attn(q, k, v, *, B, Hq, Hkv, Lq, Lk, d, dv, ldv=None, scale, causal, kv_range=None,
-         nthreads=None, elem=None, mutant: int = 0):
+         blocks=None, nthreads=None, elem=None, mutant: int = 0):
     """Full attention: O [B,Hq,Lq,dv] and LSE [B,Hq,Lq] in float64."""
     rows = np.arange(B * Hq * Lq, dtype=np.int64)
     o, lse = attn_rows(q, k, v, rows, B=B, Hq=Hq, Hkv=Hkv, Lq=Lq, Lk=Lk, d=d, dv=dv, ldv=ldv,
-                       scale=scale, causal=causal, kv_range=kv_range, nthreads=nthreads,
-                       elem=elem, mutant=mutant)
+                       scale=scale, causal=causal, kv_range=kv_range, blocks=blocks,
+                       nthreads=nthreads, elem=elem, mutant=mutant)
     return o.reshape(B, Hq, Lq, dv), lse.reshape(B, Hq, Lq)
 
 

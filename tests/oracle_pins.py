@@ -284,7 +284,109 @@ def pin_library_sdpa_f16(mutant=0):
         assert np.max(np.abs(lse - ref_l.numpy())) <= 1e-12
 
 
+def random_block_lists(B, Hq, nqb, nkb, seed, p_keep=0.5, max_blk=None):
+    """Sorted unique key-block lists per (b, h, query block), some of them empty."""
+    g = np.random.default_rng(seed)
+    max_blk = nkb if max_blk is None else max_blk
+    idx = np.full((B, Hq, nqb, max_blk), -7, dtype=np.int32)  # unused entries hold junk
+    cnt = np.zeros((B, Hq, nqb), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            for qb in range(nqb):
+                keep = np.flatnonzero(g.random(nkb) < p_keep)[:max_blk]
+                if (b + h + qb) % 5 == 3:
+                    keep = keep[:0]
+                idx[b, h, qb, :keep.size] = keep
+                cnt[b, h, qb] = keep.size
+    return idx, cnt
+
+
+def block_mask(idx, cnt, Lq, Lk, blk_q, blk_k, causal):
+    """Boolean [B, Hq, Lq, Lk] visibility mask built from block lists (and the causal rule)."""
+    B, Hq, nqb, _ = idx.shape
+    m = np.zeros((B, Hq, Lq, Lk), dtype=bool)
+    for b in range(B):
+        for h in range(Hq):
+            for qb in range(nqb):
+                for kb in idx[b, h, qb, :cnt[b, h, qb]]:
+                    m[b, h, qb * blk_q:(qb + 1) * blk_q, kb * blk_k:(kb + 1) * blk_k] = True
+    if causal:
+        m &= bottom_right_mask(Lq, Lk, True).numpy()[None, None]
+    return torch.from_numpy(m)
+
+
+SPARSE_SHAPES = [
+    # B, Hq, Hkv, Lq, Lk, d, blk_q, blk_k, causal
+    (1, 2, 1, 11, 13, 8, 4, 3, True),
+    (2, 4, 2, 9, 9, 4, 3, 2, False),
+    (1, 2, 2, 5, 12, 8, 2, 5, True),
+]
+
+
+def pin_sparse_full_lists_equal_dense(mutant=0):
+    """Listing every key block reduces block-sparse attention to the dense definition."""
+    for n, (B, Hq, Hkv, Lq, Lk, d, bq, bk, causal) in enumerate(SPARSE_SHAPES):
+        q = rnd_bf16((B, Hq, Lq, d), 300 + n)
+        k = rnd_bf16((B, Hkv, Lk, d), 310 + n)
+        v = rnd_bf16((B, Hkv, Lk, d), 320 + n)
+        nqb, nkb = -(-Lq // bq), -(-Lk // bk)
+        idx = np.tile(np.arange(nkb, dtype=np.int32), (B, Hq, nqb, 1))
+        cnt = np.full((B, Hq, nqb), nkb, dtype=np.int32)
+        a = _args(B, Hq, Hkv, Lq, Lk, d, d, causal)
+        o, l = oracle.attn(q, k, v, blocks=(idx, cnt, bq, bk), mutant=mutant, **a)
+        o2, l2 = oracle.attn(q, k, v, mutant=mutant, **a)
+        assert np.array_equal(o, o2) and np.array_equal(l, l2)
+
+
+def pin_sparse_library_sdpa(mutant=0):
+    """Random block lists against torch's fp64 SDPA with the explicit block mask; rows that see
+    no key are O = 0, LSE = -inf."""
+    for n, (B, Hq, Hkv, Lq, Lk, d, bq, bk, causal) in enumerate(SPARSE_SHAPES):
+        q = rnd_bf16((B, Hq, Lq, d), 330 + n)
+        k = rnd_bf16((B, Hkv, Lk, d), 340 + n)
+        v = rnd_bf16((B, Hkv, Lk, d), 350 + n)
+        nqb, nkb = -(-Lq // bq), -(-Lk // bk)
+        idx, cnt = random_block_lists(B, Hq, nqb, nkb, 360 + n)
+        o, lse = oracle.attn(q, k, v, blocks=(idx, cnt, bq, bk), mutant=mutant,
+                             **_args(B, Hq, Hkv, Lq, Lk, d, d, causal))
+        mask = block_mask(idx, cnt, Lq, Lk, bq, bk, causal)
+        G = Hq // Hkv
+        kr, vr = f64(k).repeat_interleave(G, 1), f64(v).repeat_interleave(G, 1)
+        s = torch.einsum("bhid,bhjd->bhij", f64(q), kr) / math.sqrt(d)
+        s = s.masked_fill(~mask, -math.inf)
+        seen = mask.any(-1).numpy()
+        assert (~seen).any() and seen.any()
+        ref_l = torch.logsumexp(s, dim=-1).numpy()
+        ref_o = torch.einsum("bhij,bhjd->bhid", torch.softmax(s, -1).nan_to_num(0.0), vr).numpy()
+        assert np.max(np.abs(o[seen] - ref_o[seen])) <= 1e-12
+        assert np.max(np.abs(lse[seen] - ref_l[seen])) <= 1e-12
+        assert np.all(o[~seen] == 0.0) and np.all(lse[~seen] == -math.inf)
+
+
+def pin_sparse_equals_merged_block_partials(mutant=0):
+    """Block-sparse O/LSE equal the log-sum-exp merge of the per-block split partials of the
+    listed blocks (each partial from the contiguous key range of one block)."""
+    B, Hq, Hkv, Lq, Lk, d, bq, bk, causal = 1, 2, 1, 8, 14, 8, 4, 4, True
+    q = rnd_bf16((B, Hq, Lq, d), 370)
+    k = rnd_bf16((B, Hkv, Lk, d), 371)
+    v = rnd_bf16((B, Hkv, Lk, d), 372)
+    nqb, nkb = -(-Lq // bq), -(-Lk // bk)
+    idx = np.full((B, Hq, nqb, 3), 0, dtype=np.int32)
+    idx[..., :] = [0, 2, 3]
+    cnt = np.full((B, Hq, nqb), 3, dtype=np.int32)
+    a = _args(B, Hq, Hkv, Lq, Lk, d, d, causal)
+    rows = np.arange(B * Hq * Lq)
+    o, l = oracle.attn_rows(q, k, v, rows, blocks=(idx, cnt, bq, bk), mutant=mutant, **a)
+    parts = [oracle.attn_rows(q, k, v, rows, kv_range=(kb * bk, min(Lk, kb * bk + bk)), mutant=mutant, **a)
+             for kb in (0, 2, 3)]
+    om, lm = oracle.combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]), mutant=mutant)
+    fin = np.isfinite(l)
+    assert np.array_equal(fin, np.isfinite(lm))
+    assert np.max(np.abs(o - om)) <= 1e-12 and np.max(np.abs(l[fin] - lm[fin])) <= 1e-12
+
+
 ALL_PINS = [pin_rows_sum_to_one, pin_transposed_flow, pin_constant_v, pin_one_hot,
             pin_closed_forms, pin_shift_invariance, pin_gqa_equals_repeated_mha,
             pin_split_merge, pin_library_sdpa, pin_latent_kv, pin_golden_worked_example,
-            pin_widen_tables, pin_library_sdpa_f16]
+            pin_widen_tables, pin_library_sdpa_f16, pin_sparse_full_lists_equal_dense,
+            pin_sparse_library_sdpa, pin_sparse_equals_merged_block_partials]
