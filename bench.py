@@ -7,8 +7,8 @@ Llama-3-8B-shaped causal GQA prefill (B=1, Hq=32, Hkv=8, L=8192, d=128): metric 
 (algorithmic flops = 2*(d+dv) per visible query/key pair). The same JSON line also carries the
 MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) and the GQA
 decode (B=16, 32 query heads on 8 kv heads, Lk=32768) measured in HBM GB/s, and the fp16-input
-variants of the prefill and of the MLA decode, each with its roofline fraction against
-MEASURED_PEAKS.json.
+variants of the prefill and of the MLA decode, and the block-sparse 128K prefill over its given
+index, each with its roofline fraction against MEASURED_PEAKS.json.
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching stream;
 L2 is flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU (torchrun):
@@ -205,6 +205,25 @@ def bench_prefill(w, dev, steps, warmup, flush, stream):
     return times, (q, k, v)
 
 
+def bench_prefill_sparse(w, dev, steps, warmup, flush, stream):
+    """Block-sparse prefill over the workload's given index (inputs.block_lists)."""
+    from exact_attention_139_b200 import attn
+    from exact_attention_139_b200.inputs import block_lists, sparse_visible_pairs
+    q, k, v = make_inputs(w)
+    idx, cnt = block_lists(w)
+    pairs = sparse_visible_pairs(w, idx, cnt)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    del q, k, v
+    idx_d, cnt_d = torch.from_numpy(idx).to(dev), torch.from_numpy(cnt).to(dev)
+    o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=w.torch_dtype, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    step = lambda: attn.attn_fwd_sparse(qd, kd, vd, idx_d, cnt_d, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    times = time_steps(step, steps, warmup, flush, stream)
+    if attn.attn_check_device() != attn.ATTN_OK:
+        raise RuntimeError("device error during the sparse prefill benchmark")
+    return times, pairs
+
+
 def bench_prefill_e2e(w, dev, steps, warmup, host):
     """End to end: pinned host inputs -> device, attn_fwd, O and LSE back to pinned host memory."""
     from exact_attention_139_b200 import attn
@@ -335,6 +354,21 @@ def run_ours(args):
                 "roofline": {"bound": "hbm", "achieved": round(dfgbs, 1), "peak": float(peaks["hbm_gbs"]),
                              "unit": "GB/s", "frac": round(dfgbs / float(peaks["hbm_gbs"]), 4)}}
             launches += args.steps + 2 * args.steps
+        if not args.no_sparse:
+            ws_ = rank_workload(WORKLOADS["sparse_prefill_128k"], rank)
+            sp_steps = max(3, args.steps // 10)  # ~11 ms per step
+            stimes, pairs = bench_prefill_sparse(ws_, dev, sp_steps, min(args.warmup, 5), flush, stream)
+            sms = max_over_ranks(sum(stimes) / len(stimes), world)
+            sflops = pairs * 2.0 * (ws_.d + ws_.dv)
+            stf = sflops / (sms * 1e-3) / 1e12
+            extras["prefill_sparse"] = {
+                "workload": ws_.name, "metric": "attention TFLOPS over the visible (listed, causal) pairs",
+                "value": round(stf * world, 2), "ms_per_step": round(sms, 4), "steps": sp_steps,
+                "density": round(pairs / ws_.visible_pairs(), 4),
+                "dense_equivalent_tflops": round(ws_.flops() / (sms * 1e-3) / 1e12, 1),
+                "roofline": {"bound": "tensor", "achieved": round(stf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": round(stf / peak_tf, 4), "algorithmic_flops_per_launch": sflops}}
+            launches += sp_steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -409,6 +443,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the decode measurement")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-f16", action="store_true", help="skip the fp16-input measurements")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

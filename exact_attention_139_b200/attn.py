@@ -7,6 +7,7 @@ library. Importing this module raises if the library has not been built; there i
 Functions keep the C names; q, k, v (and o) are all bf16 or all fp16, and the element type is
 taken from q (the C ``*_typed`` entry points receive it):
     attn_fwd(q, k, v, causal=..., scale=None, out=None, lse=None)          -> (o, lse)
+    attn_fwd_sparse(q, k, v, block_idx, block_cnt, causal=..., ...)        -> (o, lse)
     attn_decode(q, k, v, causal=..., dv=None, num_splits=0, impl=0, ...)   -> (o, lse)
     attn_combine(o_part, lse_part, out=None, lse=None, dtype=bf16)         -> (o, lse)
     attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)         -> int
@@ -33,6 +34,8 @@ _lib.attn_fwd.restype = _i
 _lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _vp]
 _lib.attn_fwd_typed.restype = _i
 _lib.attn_fwd_typed.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _i, _vp]
+_lib.attn_fwd_sparse_typed.restype = _i
+_lib.attn_fwd_sparse_typed.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _vp, _vp, _i, _i, _vp]
 _lib.attn_decode_workspace_size.restype = _sz
 _lib.attn_decode_workspace_size.argtypes = [_i] * 7
 _lib.attn_decode.restype = _i
@@ -124,6 +127,38 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
                                lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
                                scale, int(bool(causal)), code_t, _stream_handle(q.device))
     _check(code, "attn_fwd")
+    return out, lse
+
+
+SPARSE_BLOCK = 128  # query rows / keys per block of attn_fwd_sparse's index lists
+
+
+def attn_fwd_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_idx: torch.Tensor,
+                    block_cnt: torch.Tensor, *, causal: bool, scale: float | None = None,
+                    out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """Block-sparse attention: block_idx int32 [B, Hq, ceil(Lq/128), max_blocks] (sorted, distinct
+    128-key block ids per query block), block_cnt int32 [B, Hq, ceil(Lq/128)] (entries used)."""
+    code_t = _elem_code(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(block_idx, "block_idx", torch.int32)
+    _need(block_cnt, "block_cnt", torch.int32)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dv = v.shape[-1]
+    nqb = (Lq + SPARSE_BLOCK - 1) // SPARSE_BLOCK
+    if block_cnt.shape != (B, Hq, nqb) or block_idx.dim() != 4 or block_idx.shape[:3] != (B, Hq, nqb):
+        raise ValueError(f"block lists must be [B, Hq, {nqb}, max_blocks] and [B, Hq, {nqb}]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
+    _need(out, "out", q.dtype)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    code = _lib.attn_fwd_sparse_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      B, Hq, Hkv, Lq, Lk, d, dv, scale, int(bool(causal)), block_idx.data_ptr(),
+                                      block_cnt.data_ptr(), block_idx.shape[3], code_t, _stream_handle(q.device))
+    _check(code, "attn_fwd_sparse")
     return out, lse
 
 

@@ -21,7 +21,7 @@ namespace {
 
 using attn::DecodeParams;
 
-constexpr int kAbiVersion = 10100;  // 1.1.0: element-type (*_typed) entry points
+constexpr int kAbiVersion = 10200;  // 1.2.0: block-sparse forward (attn_fwd_sparse_typed)
 
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -337,9 +337,16 @@ attn_status with_elem(int dtype, Fn&& fn) {
   return ATTN_ERR_INVALID_ARG;
 }
 
-template <typename E>
+// Block lists of the sparse mode (all nullptr / 0 in dense mode).
+struct SparseBlocks {
+  const int32_t* idx;
+  const int32_t* cnt;
+  int max_blk;
+};
+
+template <typename E, bool SPARSE>
 attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
-                     int Lk, int d, float scale, int causal, void* stream) {
+                     int Lk, int d, float scale, int causal, SparseBlocks sb, void* stream) {
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int n_qtiles = (Lq + 127) / 128;
   CUtensorMap tq, tk, tv;
@@ -366,16 +373,21 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   p.group_b = (int)std::max(1LL, std::min<long long>(B, (64LL << 20) / std::max(1LL, kv_per_batch)));
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.blk_idx = sb.idx;
+  p.blk_cnt = sb.cnt;
+  p.max_blk = sb.max_blk;
+  p.n_qblocks = n_qtiles;
+  p.n_kblocks = (Lk + 127) / 128;
   // persistent grid: one CTA per SM (fewer when there are fewer work units)
   const int grid = (int)std::min<long long>(units, current_sm_count());
   if (d == 128) {
     using C = attn::Prefill2Cfg<128>;
-    if (!allow_smem(attn::prefill2_kernel<128, E>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<128, E><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    if (!allow_smem(attn::prefill2_kernel<128, E, SPARSE>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<128, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   } else {
     using C = attn::Prefill2Cfg<64>;
-    if (!allow_smem(attn::prefill2_kernel<64, E>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<64, E><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    if (!allow_smem(attn::prefill2_kernel<64, E, SPARSE>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    attn::prefill2_kernel<64, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
   }
   return launch_status();
 }
@@ -468,7 +480,26 @@ attn_status attn_fwd_typed(const void* q, const void* k, const void* v, void* o,
   if (st != ATTN_OK) return st;
   if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
   return with_elem(dtype, [&](auto e) {
-    return fwd_impl<decltype(e)>(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal, stream);
+    return fwd_impl<decltype(e), false>(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal,
+                                        SparseBlocks{nullptr, nullptr, 0}, stream);
+  });
+}
+
+attn_status attn_fwd_sparse_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                                  int Hkv, int Lq, int Lk, int d, int dv, float scale, int causal,
+                                  const int32_t* block_idx, const int32_t* block_cnt, int max_blocks, int dtype,
+                                  void* stream) {
+  if (!valid_dtype(dtype)) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (!block_idx || !block_cnt || max_blocks < 1) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(block_idx, 4) || !aligned(block_cnt, 4)) return ATTN_ERR_MISALIGNED;
+  if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+  const long long n_lists = (long long)B * Hq * ((Lq + 127) / 128);
+  if (n_lists * max_blocks > (1LL << 40)) return ATTN_ERR_UNSUPPORTED;
+  return with_elem(dtype, [&](auto e) {
+    return fwd_impl<decltype(e), true>(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal,
+                                       SparseBlocks{block_idx, block_cnt, max_blocks}, stream);
   });
 }
 
@@ -611,13 +642,16 @@ attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
 
 attn_status attn_check_device(void* stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
-  unsigned int word = 0;
+  unsigned int word = 0, input_word = 0;
   if (cudaMemcpyFromSymbol(&word, attn::g_attn_dev_error, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (word != 0) {
-    const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(attn::g_attn_dev_error, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-    return ATTN_ERR_TIMEOUT;
-  }
+  if (cudaMemcpyFromSymbol(&input_word, attn::g_attn_dev_input_error, sizeof(input_word)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (word != 0 && cudaMemcpyToSymbol(attn::g_attn_dev_error, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (input_word != 0 && cudaMemcpyToSymbol(attn::g_attn_dev_input_error, &zero, sizeof(zero)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (word != 0) return ATTN_ERR_TIMEOUT;
+  if (input_word != 0) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 

@@ -38,6 +38,11 @@ struct Prefill2Params {
   int group_b;  // batches per scheduling group (their K/V fits comfortably in L2)
   int causal;
   float scale_log2;
+  // block-sparse mode only: per (batch, head, 128-row query block) a sorted list of distinct
+  // 128-key blocks; cnt [B, Hq, n_qblocks], idx [B, Hq, n_qblocks, max_blk]
+  const int32_t* blk_idx;
+  const int32_t* blk_cnt;
+  int max_blk, n_qblocks, n_kblocks;
 };
 
 #ifndef ATTN_EXP2_EMULATE_MASK
@@ -86,6 +91,81 @@ struct UnitCoords {
   int b, h, q0;
 };
 
+// The key blocks one query tile processes, in increasing order: 0 .. n-1 in dense mode, the
+// caller's list in block-sparse mode.
+struct TileList {
+  const int32_t* idx;  // nullptr: dense
+  int n;
+  __device__ __forceinline__ int block(int t) const { return idx ? __ldg(idx + t) : t; }
+};
+
+// Tile x (0: rows q0.., 1: rows q0 + 128..) of unit uc. In block-sparse mode the list is read
+// up to its first entry that is out of range or not above its predecessor (the kernel then
+// records kDevErrBadIndex when `report`) and stops before the first block that lies wholly
+// above the causal diagonal of the tile: every later entry would be masked out too.
+template <bool SPARSE>
+__device__ __forceinline__ TileList prefill_tile_list(const Prefill2Params& p, const UnitCoords& uc, int x,
+                                                      bool report) {
+  const int qr0 = uc.q0 + 128 * x;
+  const int n_dense = prefill_kv_tiles(p, qr0);
+  if constexpr (!SPARSE) {
+    return TileList{nullptr, n_dense};
+  } else {
+    if (n_dense == 0) return TileList{nullptr, 0};
+    const long long slot = ((long long)uc.b * p.Hq + uc.h) * p.n_qblocks + qr0 / 128;
+    const int32_t* lst = p.blk_idx + slot * p.max_blk;
+    int cnt = __ldg(p.blk_cnt + slot);
+    bool bad = cnt < 0 || cnt > p.max_blk;
+    if (bad) cnt = 0;
+    int n = 0, prev = -1;
+    for (int t = 0; t < cnt; ++t) {
+      const int kb = __ldg(lst + t);
+      if (kb <= prev || kb >= p.n_kblocks) {
+        bad = true;
+        break;
+      }
+      if (kb >= n_dense) break;
+      prev = kb;
+      ++n;
+    }
+    if (bad && report) raise_bad_index();
+    return TileList{lst, n};
+  }
+}
+
+// Walks the union of the two tiles' block lists in increasing order. Every role of the CTA (TMA
+// producer, MMA issuer, softmax warpgroups) derives the same sequence from the same lists.
+struct UnionWalk {
+  TileList a, b;
+  int ia, ib;
+  __device__ __forceinline__ UnionWalk(const TileList& la, const TileList& lb) : a(la), b(lb), ia(0), ib(0) {}
+  // Next block of the union and which tiles list it; false once both lists are exhausted.
+  __device__ __forceinline__ bool next(int& kb, bool& in_a, bool& in_b) {
+    const int ka = ia < a.n ? a.block(ia) : 0x7fffffff;
+    const int kc = ib < b.n ? b.block(ib) : 0x7fffffff;
+    if (ka == 0x7fffffff && kc == 0x7fffffff) return false;
+    kb = min(ka, kc);
+    in_a = ka == kb;
+    in_b = kc == kb;
+    ia += in_a ? 1 : 0;
+    ib += in_b ? 1 : 0;
+    return true;
+  }
+};
+
+template <bool SPARSE>
+__device__ __forceinline__ int union_size(const TileList& la, const TileList& lb) {
+  if constexpr (!SPARSE) {
+    return max(la.n, lb.n);
+  } else {
+    UnionWalk w(la, lb);
+    int n = 0, kb;
+    bool x0, x1;
+    while (w.next(kb, x0, x1)) ++n;
+    return n;
+  }
+}
+
 // Unit order. Batches are taken in groups of group_b whose K/V together fits in L2 with room to
 // spare; within a group the units are sorted by cost (heaviest query-tile pair first: under a
 // causal mask the cost of a pair grows with its position), then by batch, then by head, so that
@@ -116,7 +196,7 @@ __device__ __forceinline__ int prefill_unit_index(int k, int cta, int grid) {
   return k * grid + ((k & 1) ? grid - 1 - cta : cta);
 }
 
-template <int D, typename E>
+template <int D, typename E, bool SPARSE>
 __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Prefill2Params p) {
@@ -186,23 +266,50 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           tma_load_3d(dst + C::KV_BYTES + c * C::CHUNK, &tm_v, full, 64 * c, tile * C::BN, zkv);
         ++kv_t;
       };
-      for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
-        const UnitCoords uc = prefill_unit(p, u);
-        const int nA = prefill_kv_tiles(p, uc.q0), nB = prefill_kv_tiles(p, uc.q0 + 128);
-        const int n = max(nA, nB);
-        if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
-        if (!ok) break;
-        const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
-        mbar_arrive_expect_tx(bar_q_full, (nB > 0 ? 2 : 1) * C::Q_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
-        if (nB > 0) {
-#pragma unroll
-          for (int c = 0; c < C::DC; ++c)
-            tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+      if constexpr (SPARSE) {
+        for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
+          const UnitCoords uc = prefill_unit(p, u);
+          const TileList la = prefill_tile_list<SPARSE>(p, uc, 0, true);
+          const TileList lb = prefill_tile_list<SPARSE>(p, uc, 1, true);
+          if (la.n == 0 && lb.n == 0) continue;  // nothing to load: the softmax writes the empty rows
+          if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
+          if (!ok) break;
+          const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
+          mbar_arrive_expect_tx(bar_q_full, ((la.n > 0 ? 1 : 0) + (lb.n > 0 ? 1 : 0)) * C::Q_BYTES);
+          if (la.n > 0) {
+  #pragma unroll
+            for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
+          }
+          if (lb.n > 0) {
+  #pragma unroll
+            for (int c = 0; c < C::DC; ++c)
+              tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+          }
+          ++qc;
+          UnionWalk walk(la, lb);
+          int kb;
+          bool in_a, in_b;
+          while (ok && walk.next(kb, in_a, in_b)) load_kv(kb, zkv);
         }
-        ++qc;
-        for (int j = 0; j < n && ok; ++j) load_kv(j, zkv);
+      } else {
+        for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
+          const UnitCoords uc = prefill_unit(p, u);
+          const int nA = prefill_kv_tiles(p, uc.q0), nB = prefill_kv_tiles(p, uc.q0 + 128);
+          const int n = max(nA, nB);
+          if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
+          if (!ok) break;
+          const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
+          mbar_arrive_expect_tx(bar_q_full, (nB > 0 ? 2 : 1) * C::Q_BYTES);
+  #pragma unroll
+          for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
+          if (nB > 0) {
+  #pragma unroll
+            for (int c = 0; c < C::DC; ++c)
+              tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+          }
+          ++qc;
+          for (int j = 0; j < n && ok; ++j) load_kv(j, zkv);
+        }
       }
       if (!ok) {
         if (qc > 0) mbar_wait_drain(bar_q_full, (qc - 1) & 1);
@@ -237,63 +344,136 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       // product of tile j+1 is the one on P: the stage of tile j is released right after its
       // last P.V product (one commit, while the tensor core still has S work queued), and the
       // stage of tile j+1 is awaited before the first S of tile j+1.
-      for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
-        const UnitCoords uc = prefill_unit(p, u);
-        int nX[2];
-        nX[0] = prefill_kv_tiles(p, uc.q0);
-        nX[1] = prefill_kv_tiles(p, uc.q0 + 128);
-        const int n = max(nX[0], nX[1]);
-        ok = mbar_wait(bar_q_full, qc & 1, 63);
-        if (!ok) break;
-        ++qc;
-        tc_fence_after();
-        wait_stage(kv_t, 64);  // K_0, V_0
-        if (!ok) break;
-        for (int x = 0; x < 2; ++x)
-          if (nX[x] > 0) issue_s(x, kv_t);
-        if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
-        for (int j = 0; j < n && ok; ++j) {
-          const int si = kv_t + j;                // stage of tile j
-          const int x_last = (j < nX[1]) ? 1 : 0;  // last tile whose P.V reads V_j
-          bool next_ready = false;
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (j >= nX[x]) continue;
-            if (j == 0 && units_done[x] > 0) {
-              ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
-              if (!ok) break;
-            }
-            ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
-            if (!ok) break;
-            ++p_cnt[x];
-            tc_fence_after();
-            const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < C::BN / 16; ++kk) {
-              const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
-              // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
-              mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            // K_j was last read by S of tile j (issued earlier), V_j by this product
-            if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
-            if (j + 1 < nX[x]) {
-              if (!next_ready) {
-                wait_stage(si + 1, 68);  // K_{j+1}, V_{j+1}
+      if constexpr (SPARSE) {
+        for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
+          const UnitCoords uc = prefill_unit(p, u);
+          const TileList lx[2] = {prefill_tile_list<SPARSE>(p, uc, 0, false), prefill_tile_list<SPARSE>(p, uc, 1, false)};
+          if (lx[0].n == 0 && lx[1].n == 0) continue;
+          const int n = union_size<SPARSE>(lx[0], lx[1]);  // key blocks loaded for this unit
+          ok = mbar_wait(bar_q_full, qc & 1, 63);
+          if (!ok) break;
+          ++qc;
+          tc_fence_after();
+          UnionWalk walk(lx[0], lx[1]);
+          int kb;
+          bool in[2];
+          walk.next(kb, in[0], in[1]);
+          wait_stage(kv_t, 64);  // K, V of the first block
+          if (!ok) break;
+          for (int x = 0; x < 2; ++x)
+            if (in[x]) issue_s(x, kv_t);
+          if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
+          int jx[2] = {0, 0};                    // blocks of each tile already multiplied by V
+          for (int j = 0; j < n && ok; ++j) {
+            const int si = kv_t + j;  // stage of union block j
+            bool in_next[2] = {false, false};
+            const bool has_next = j + 1 < n && walk.next(kb, in_next[0], in_next[1]);
+            const int x_last = in[1] ? 1 : 0;  // last tile whose P.V reads this V
+            bool next_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+              if (in[x]) {
+                if (jx[x] == 0 && units_done[x] > 0) {
+                  ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
+                  if (!ok) break;
+                }
+                ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
                 if (!ok) break;
-                next_ready = true;
+                ++p_cnt[x];
+                tc_fence_after();
+                const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
+  #pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                  const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
+                  // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
+                  mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (jx[x] > 0 || kk > 0) ? 1u : 0u);
+                }
+                // K was last read by the S products of this block (issued earlier), V by this one
+                if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
               }
-              issue_s(x, si + 1);
+              if (has_next && in_next[x]) {
+                if (!next_ready) {
+                  wait_stage(si + 1, 68);  // K, V of the next union block
+                  if (!ok) break;
+                  next_ready = true;
+                }
+                issue_s(x, si + 1);
+              }
+              if (in[x]) {
+                if (jx[x] == lx[x].n - 1) {
+                  mma_commit(bar_o_ready + 8 * x);
+                  ++units_done[x];
+                }
+                ++jx[x];
+              }
             }
-            if (j == nX[x] - 1) {
-              mma_commit(bar_o_ready + 8 * x);
-              ++units_done[x];
-            }
+            if (!ok) break;
+            // Q may be reloaded once the last S of this unit (issued in step n-2) is done
+            if (j == n - 2) mma_commit(bar_q_empty);
+            in[0] = in_next[0];
+            in[1] = in_next[1];
           }
           if (!ok) break;
-          // Q may be reloaded once the last S of this unit (issued in iteration n-2) is done
-          if (j == n - 2) mma_commit(bar_q_empty);
+          kv_t += n;
         }
-        if (!ok) break;
-        kv_t += n;
+      } else {
+        for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
+          const UnitCoords uc = prefill_unit(p, u);
+          int nX[2];
+          nX[0] = prefill_kv_tiles(p, uc.q0);
+          nX[1] = prefill_kv_tiles(p, uc.q0 + 128);
+          const int n = max(nX[0], nX[1]);
+          ok = mbar_wait(bar_q_full, qc & 1, 63);
+          if (!ok) break;
+          ++qc;
+          tc_fence_after();
+          wait_stage(kv_t, 64);  // K_0, V_0
+          if (!ok) break;
+          for (int x = 0; x < 2; ++x)
+            if (nX[x] > 0) issue_s(x, kv_t);
+          if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
+          for (int j = 0; j < n && ok; ++j) {
+            const int si = kv_t + j;                // stage of tile j
+            const int x_last = (j < nX[1]) ? 1 : 0;  // last tile whose P.V reads V_j
+            bool next_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+              if (j >= nX[x]) continue;
+              if (j == 0 && units_done[x] > 0) {
+                ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
+                if (!ok) break;
+              }
+              ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
+              if (!ok) break;
+              ++p_cnt[x];
+              tc_fence_after();
+              const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
+  #pragma unroll
+              for (int kk = 0; kk < C::BN / 16; ++kk) {
+                const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
+                // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
+                mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+              }
+              // K_j was last read by S of tile j (issued earlier), V_j by this product
+              if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
+              if (j + 1 < nX[x]) {
+                if (!next_ready) {
+                  wait_stage(si + 1, 68);  // K_{j+1}, V_{j+1}
+                  if (!ok) break;
+                  next_ready = true;
+                }
+                issue_s(x, si + 1);
+              }
+              if (j == nX[x] - 1) {
+                mma_commit(bar_o_ready + 8 * x);
+                ++units_done[x];
+              }
+            }
+            if (!ok) break;
+            // Q may be reloaded once the last S of this unit (issued in iteration n-2) is done
+            if (j == n - 2) mma_commit(bar_q_empty);
+          }
+          if (!ok) break;
+          kv_t += n;
+        }
       }
       if (!ok && issued) {
         mma_commit(bar_drain);
@@ -313,9 +493,20 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
       const UnitCoords uc = prefill_unit(p, u);
       const int qx0 = uc.q0 + 128 * x;
-      const int nt = prefill_kv_tiles(p, qx0);
-      if (nt == 0) continue;
+      if (qx0 >= p.Lq) continue;  // tile past the last query row
+      const TileList lst = prefill_tile_list<SPARSE>(p, uc, x, false);
+      const int nt = lst.n;
       const int row = qx0 + r;
+      if (SPARSE && nt == 0) {
+        // no listed block: these rows see no key (O = 0, LSE = -inf); nothing was loaded for them
+        if (row < p.Lq) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + row) * D);
+#pragma unroll
+          for (int q = 0; q < D / 8; ++q) dst[q] = make_uint4(0u, 0u, 0u, 0u);
+          if (p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = -INFINITY;
+        }
+        continue;
+      }
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
         ok = mbar_wait(bar_s_full + 8 * x, s_cnt & 1, 69);
@@ -327,7 +518,8 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tw + s_col + 32 * c4, s[c4]);
         tmem_wait_ld();
-        const int kv0 = j * C::BN;
+        int kv0 = j * C::BN;
+        if constexpr (SPARSE) kv0 = lst.block(j) * C::BN;
         if (kv0 + C::BN > p.Lk || (p.causal && kv0 + C::BN - 1 > qx0 + off)) {
           int lim = p.Lk - 1;
           if (p.causal) lim = min(lim, row + off);
@@ -414,7 +606,8 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       if (!ok) break;
       ++o_cnt;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      float inv_l = 1.f / l;
+      if constexpr (SPARSE) inv_l = l > 0.f ? inv_l : 0.f;  // l = 0: the row saw no key
       const bool in_range = row < p.Lq;
       uint16_t* orow = p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + (in_range ? row : 0)) * D;
 #pragma unroll
@@ -432,7 +625,11 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
                                 E::pack2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
         }
       }
-      if (in_range && p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = (m_used + log2f(l)) * kLn2;
+      if (in_range && p.lse != nullptr) {
+        float lse_row = (m_used + log2f(l)) * kLn2;
+        if constexpr (SPARSE) lse_row = l > 0.f ? lse_row : -INFINITY;
+        p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = lse_row;
+      }
       tc_fence_before();
       mbar_arrive(bar_o_free + 8 * x);
     }

@@ -19,6 +19,7 @@ namespace attn {
 __device__ unsigned int g_attn_dev_error;
 
 constexpr unsigned int kDevErrTimeout = 1u;
+constexpr unsigned int kDevErrBadIndex = 2u;  // a caller-given index list broke its contract
 // Online softmax: the exponent reference only moves when a tile's max exceeds it by more than
 // this many log2 units (lazy rescaling); results are unchanged, p stays below 2^8.
 constexpr float kRescaleLog2 = 8.0f;
@@ -38,6 +39,13 @@ __device__ __forceinline__ bool dev_error_set() {
 __device__ __forceinline__ void raise_timeout(unsigned int site) {
   atomicOr(&g_attn_dev_error, kDevErrTimeout | ((site & 0xffu) << 8));
 }
+
+// Input errors found on the device (a caller-given index list that breaks its contract) go to
+// their own word: the waits do not watch it, so the kernel finishes on the lists as truncated at
+// the offending entry (every role of a CTA truncates them the same way) and the host reports it.
+__device__ unsigned int g_attn_dev_input_error;
+
+__device__ __forceinline__ void raise_bad_index() { atomicOr(&g_attn_dev_input_error, kDevErrBadIndex); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -409,7 +417,8 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t xv) {
   // is n in the exponent field
   const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
   const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-  return f2_pack(r0, r1);
+  // below the clamp (masked scores are -inf) the result is exactly 0, like ex2.approx's
+  return f2_pack(x0 < -126.f ? 0.f : r0, x1 < -126.f ? 0.f : r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -19,6 +19,11 @@ Workloads (the shapes of the pages' settings; no dataset or model weights are us
   * ``gqa_decode_32k``: GQA decode with a dense V, B=16, Hq=32, Hkv=8, Lq=1, Lk=32768,
     d=dv=128 (the batch 8-16 regime of the "Flash Attention en Modelos Pequenos" notes on the
     Llama-3-8B head shape).
+  * ``sparse_prefill_128k``: the 128K vertical-bias prefill with a given block-sparse index
+    (``block_lists``): every 128-row query block sees the first key block, a local window of
+    16 blocks ending at its diagonal block, and the blocks that hold its kv head's biased
+    "vertical" keys (the A-shape and vertical-bar patterns of the MInference article, at block
+    granularity). The index is an input here; building one from attention scores is not.
 """
 from __future__ import annotations
 
@@ -46,6 +51,7 @@ class Workload:
     vertical_bias: float = 0.0
     seed: int = BASE_SEED
     dtype: str = "bf16"           # element type of q, k, v and o: "bf16" or "f16"
+    sparse_window: int = 0        # > 0: block-sparse index with a local window of this many blocks
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -97,7 +103,64 @@ WORKLOADS = {
                                   vertical_keys=64, vertical_bias=2.0, seed=BASE_SEED + 5),
     "gqa_decode_32k": Workload("gqa_decode_32k", 16, 32, 8, 1, 32768, 128, 128, True,
                                seed=BASE_SEED + 6),
+    "sparse_prefill_128k": Workload("sparse_prefill_128k", 1, 32, 8, 131072, 131072, 128, 128, True,
+                                    vertical_keys=64, vertical_bias=2.0, seed=BASE_SEED + 5,
+                                    sparse_window=16),
 }
+
+SPARSE_BLOCK = 128
+
+
+def block_lists(w: Workload):
+    """(idx, cnt) int32 numpy arrays [B, Hq, nqb, max] / [B, Hq, nqb] of the block-sparse index of
+    ``w``: for query block qb of head (b, h), the sorted distinct key blocks {0}, the window
+    qb - sparse_window + 1 .. qb (shifted by the causal offset), and the blocks holding the
+    vertical keys of kv head h // (Hq / Hkv), each kept only when at or below the diagonal."""
+    import numpy as np
+    nqb = -(-w.Lq // SPARSE_BLOCK)
+    nkb = -(-w.Lk // SPARSE_BLOCK)
+    off_blocks = (w.Lk - w.Lq) // SPARSE_BLOCK
+    pos = vertical_positions(w)
+    G = w.Hq // w.Hkv
+    lists = {}
+    for b in range(w.B):
+        for hk in range(w.Hkv):
+            vb = np.unique(pos[b * w.Hkv + hk].numpy() // SPARSE_BLOCK) if pos else np.zeros(0, np.int64)
+            for qb in range(nqb):
+                diag = min(nkb - 1, qb + off_blocks) if w.causal else nkb - 1
+                s = {0} | set(range(max(0, diag - w.sparse_window + 1), diag + 1))
+                s |= {int(x) for x in vb if x <= diag}
+                lists[(b, hk, qb)] = sorted(s)
+    max_len = max(len(v) for v in lists.values())
+    idx = np.zeros((w.B, w.Hq, nqb, max_len), dtype=np.int32)
+    cnt = np.zeros((w.B, w.Hq, nqb), dtype=np.int32)
+    for (b, hk, qb), lst in lists.items():
+        for h in range(hk * G, (hk + 1) * G):
+            idx[b, h, qb, :len(lst)] = lst
+            cnt[b, h, qb] = len(lst)
+    return idx, cnt
+
+
+def sparse_visible_pairs(w: Workload, idx, cnt) -> int:
+    """(query row, key) pairs inside the listed blocks that the causal mask keeps."""
+    import numpy as np
+    nqb = idx.shape[2]
+    nkb = -(-w.Lk // SPARSE_BLOCK)
+    off = w.Lk - w.Lq
+    kstart = np.arange(nkb) * SPARSE_BLOCK
+    kend = np.minimum(kstart + SPARSE_BLOCK, w.Lk)
+    total = 0
+    for qb in range(nqb):
+        rows = np.arange(qb * SPARSE_BLOCK, min(w.Lq, (qb + 1) * SPARSE_BLOCK))
+        if w.causal:
+            last = np.minimum(rows[:, None] + off, kend[None, :] - 1)
+            per_kb = np.clip(last - kstart[None, :] + 1, 0, None).sum(axis=0)
+        else:
+            per_kb = (kend - kstart) * rows.size
+        for b in range(w.B):
+            for h in range(w.Hq):
+                total += int(per_kb[idx[b, h, qb, :cnt[b, h, qb]]].sum())
+    return total
 
 
 def _planes(g: torch.Generator, lead: int, rows: int, cols: int, dtype=torch.bfloat16) -> torch.Tensor:

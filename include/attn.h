@@ -35,6 +35,8 @@
  *    with nothing enqueued. A failed launch returns ATTN_ERR_CUDA. Kernels bound every wait
  *    on the GPU; a wait that runs out records ATTN_ERR_TIMEOUT in a device-side word that
  *    attn_check_device() reads (and clears); the kernel then stops early without hanging.
+ *    Device-side index lists (attn_fwd_sparse_typed) that break their contract are recorded in
+ *    a second device word (the kernel still finishes) and reported as ATTN_ERR_INVALID_ARG.
  *  - Thread safety: entry points keep no host state between calls except a once-per-process
  *    lookup of the driver's tensor-map encoder; concurrent calls on different streams are safe.
  */
@@ -91,6 +93,33 @@ attn_status attn_fwd(const void *q, const void *k, const void *v, void *o, float
 attn_status attn_fwd_typed(const void *q, const void *k, const void *v, void *o, float *lse,
                            int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, float scale,
                            int causal, int dtype, void *stream);
+
+/*
+ * attn_fwd_sparse_typed -- block-sparse forward attention over caller-given index lists.
+ *
+ * The MInference article (7minutos.es, on sparse attention for long-context prefill) describes
+ * attention weights that concentrate on a few structured regions (A-shape, vertical bars,
+ * sparse blocks) and a prefill that computes only those regions from an index built per input.
+ * This entry point takes such an index as given (building it is not part of this library) and
+ * computes the exact softmax attention restricted to it:
+ *   query rows are cut into blocks of 128 rows, keys into blocks of 128 keys; query block qb of
+ *   head (b, h) sees the keys of the blocks listed in
+ *       block_idx[((b * Hq + h) * nqb + qb) * max_blocks + t],  t < block_cnt[(b * Hq + h) * nqb + qb]
+ *   (nqb = ceil(Lq / 128)), intersected with the causal mask when causal != 0. Each list must be
+ *   strictly increasing with entries in [0, ceil(Lk / 128)); entries past the count are ignored.
+ *   A row that sees no key gets O = 0 and LSE = -inf. An A-shape pattern is the list {0} plus
+ *   the blocks of a local window; block-sparse patterns list their blocks directly.
+ *   block_idx, block_cnt  DEVICE int32 arrays owned by the caller, 4-byte aligned, read-only.
+ * Other arguments, layouts and supported shapes are those of attn_fwd_typed. A list that breaks
+ * its contract is read up to the offending entry (the kernel completes on the truncated list and
+ * nothing outside the arrays is read) and recorded on the device: attn_check_device() then
+ * returns ATTN_ERR_INVALID_ARG.
+ */
+attn_status attn_fwd_sparse_typed(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv,
+                                  float scale, int causal, const int32_t *block_idx,
+                                  const int32_t *block_cnt, int max_blocks, int dtype,
+                                  void *stream);
 
 /*
  * attn_decode_workspace_size -- bytes of device workspace attn_decode needs for the given
@@ -197,8 +226,9 @@ int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, in
 
 /*
  * attn_check_device -- synchronises `stream`, then reads and clears the device-side error
- * word that kernels set when a bounded wait runs out. Returns ATTN_OK, ATTN_ERR_TIMEOUT or
- * ATTN_ERR_CUDA (a sticky CUDA error from earlier work). For tests and diagnostics; the
+ * word that kernels set when a bounded wait runs out or a device index list is invalid. Returns
+ * ATTN_OK, ATTN_ERR_TIMEOUT, ATTN_ERR_INVALID_ARG (bad index list) or ATTN_ERR_CUDA (a sticky
+ * CUDA error from earlier work). For tests and diagnostics; the
  * compute entry points never synchronise.
  */
 attn_status attn_check_device(void *stream);
@@ -215,8 +245,9 @@ attn_status attn_selftest_wait_timeout(unsigned int limit_us, void *stream);
 /*
  * attn_selftest_exp2 -- diagnostic: y[i] = 2^x[i] for n device floats, computed with the FMA-pipe
  * polynomial the prefill softmax uses for part of its exponentials (round-to-nearest range
- * reduction, degree-3 minimax polynomial; relative error below 1e-4 for x in [-125, 64]; below -125 the results are
- * under 2^-124 but not accurate).
+ * reduction, degree-3 minimax polynomial; relative error below 1e-4 for x in [-125, 64]; for x
+ * below -126, -inf included, the result is exactly 0; between -126 and -125 it is tiny but not
+ * accurate).
  * x and y are device pointers; enqueued on `stream`.
  */
 attn_status attn_selftest_exp2(const float *x, float *y, int n, void *stream);

@@ -68,7 +68,7 @@ def test_status_strings(lib):
         seen.add(s)
     assert len(seen) == 7
     assert lib.attn_status_string(99).decode() == "unknown status"
-    assert lib.attn_abi_version() == 10100
+    assert lib.attn_abi_version() == 10200
 
 
 def fwd(lib, q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128, scale=0.1,
@@ -202,3 +202,25 @@ def test_default_workspace_covers_default_splits(lib):
         assert 1 <= s <= 256
         assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, 0) >= \
             lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, s)
+
+
+def test_sparse_argument_checks(lib):
+    """Every call below fails a host check: nothing is launched with the fake addresses."""
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.attn_fwd_sparse_typed.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp, vp, i, i, vp]
+
+    def sp(**kw):
+        a = dict(q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=256, Lk=256, d=128, dv=128,
+                 scale=0.1, causal=1, idx=0x50000, cnt=0x60000, max_blocks=2, dtype=0)
+        a.update(kw)
+        return lib.attn_fwd_sparse_typed(*a.values(), None)
+
+    assert sp(idx=None) == INVALID
+    assert sp(cnt=None) == INVALID
+    assert sp(max_blocks=0) == INVALID
+    assert sp(dtype=3) == INVALID
+    assert sp(Hq=3, Hkv=2) == INVALID
+    assert sp(idx=0x50002) == MISALIGNED
+    assert sp(cnt=0x60001) == MISALIGNED
+    assert sp(d=96, dv=96) == UNSUPPORTED
+    assert sp(q=A + 8) == MISALIGNED

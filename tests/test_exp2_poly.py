@@ -64,5 +64,10 @@ def test_device_matches_cuda_exp2(cuda_device):
     inside = torch.cat([torch.arange(1 << 20), torch.tensor([(1 << 20) + 2, (1 << 20) + 3, (1 << 20) + 4])]).to(cuda_device)
     rel = ((y[inside].double() / ref[inside].double()) - 1).abs().max().item()
     assert rel < 1e-4
-    below = y[(1 << 20):(1 << 20) + 2]  # x = -300 and -127.5: only smallness is promised
-    assert (below >= 0).all() and (below < 2.0 ** -124).all()
+    below = y[(1 << 20):(1 << 20) + 2]  # x = -300 and -127.5: below the range the result is 0
+    assert (below == 0).all()
+    lo = torch.tensor([-float("inf"), -126.5, -1000.0], device=cuda_device)
+    ylo = torch.empty_like(lo)
+    assert lib.attn_selftest_exp2(lo.data_ptr(), ylo.data_ptr(), 3, torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert (ylo == 0).all()  # masked scores (-inf) give exactly zero weight
