@@ -151,6 +151,17 @@ def rank_workload(w, rank: int):
     return w if rank == 0 else w.with_(seed=w.seed + 1000 * rank)
 
 
+def job_workload(w, world: int, rank: int, shard: str):
+    """This rank's part of the job: its own batch of the full shape (shard == "batch", weak
+    scaling), or its head shard of one layer (shard == "heads", strong scaling: Hq / world query
+    heads and the kv heads they read, replicated where a group spans ranks)."""
+    if shard == "batch" or world == 1:
+        return rank_workload(w, rank)
+    from exact_attention_139_b200.shard import head_shard
+    sh = head_shard(w.Hq, w.Hkv, world, rank)
+    return w.with_(Hq=sh.Hq, Hkv=sh.Hkv, seed=w.seed + 1000 * rank)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -276,7 +287,7 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    w = rank_workload(WORKLOADS[args.workload], rank)
+    w = job_workload(WORKLOADS[args.workload], world, rank, args.shard)
     stream = torch.cuda.current_stream(dev)
     flush = Flusher(dev)
     clocks = ClockSampler(torch.cuda.current_device())
@@ -303,14 +314,14 @@ def run_ours(args):
     del host
     launches = args.steps  # one prefill kernel per step
     if not args.no_extras:
-        wd = rank_workload(WORKLOADS["mla_decode_64k"], rank)
+        wd = job_workload(WORKLOADS["mla_decode_64k"], world, rank, args.shard)
         clocks_d = ClockSampler(torch.cuda.current_device())
         clocks_d.start()
         dtimes, splits = bench_decode(wd, dev, args.steps, args.warmup, flush, stream)
         dclk = clocks_d.stop()
         dms = max_over_ranks(sum(dtimes) / len(dtimes), world)
         gbs = wd.kv_bytes() / (dms * 1e-3) / 1e9
-        wg = rank_workload(WORKLOADS["gqa_decode_32k"], rank)
+        wg = job_workload(WORKLOADS["gqa_decode_32k"], world, rank, args.shard)
         gtimes, gsplits = bench_decode(wg, dev, args.steps, args.warmup, flush, stream)
         gms = max_over_ranks(sum(gtimes) / len(gtimes), world)
         ggbs = wg.kv_bytes() / (gms * 1e-3) / 1e9
@@ -334,7 +345,7 @@ def run_ours(args):
         if not args.no_f16:
             # fp16 inputs: same kernels with the fp16 operand format; fp16 and bf16 share one
             # nominal tensor rate on B200, so the measured bf16 peak is the fp16 denominator
-            wf = rank_workload(WORKLOADS[args.workload].with_(dtype="f16"), rank)
+            wf = job_workload(WORKLOADS[args.workload].with_(dtype="f16"), world, rank, args.shard)
             ftimes, _ = bench_prefill(wf, dev, args.steps, args.warmup, flush, stream)
             fms = max_over_ranks(sum(ftimes) / len(ftimes), world)
             ftf = wf.flops() / (fms * 1e-3) / 1e12
@@ -344,7 +355,7 @@ def run_ours(args):
                 "roofline": {"bound": "tensor", "achieved": round(ftf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                              "frac": round(ftf / peak_tf, 4),
                              "peak_source": f"{peak_src} bf16_tflops (burst) x 1 (fp16:bf16 nominal ratio)"}}
-            wdf = rank_workload(WORKLOADS["mla_decode_64k"].with_(dtype="f16"), rank)
+            wdf = job_workload(WORKLOADS["mla_decode_64k"].with_(dtype="f16"), world, rank, args.shard)
             dftimes, dfsplits = bench_decode(wdf, dev, args.steps, args.warmup, flush, stream)
             dfms = max_over_ranks(sum(dftimes) / len(dftimes), world)
             dfgbs = wdf.kv_bytes() / (dfms * 1e-3) / 1e9
@@ -355,7 +366,7 @@ def run_ours(args):
                              "unit": "GB/s", "frac": round(dfgbs / float(peaks["hbm_gbs"]), 4)}}
             launches += args.steps + 2 * args.steps
         if not args.no_sparse:
-            ws_ = rank_workload(WORKLOADS["sparse_prefill_128k"], rank)
+            ws_ = job_workload(WORKLOADS["sparse_prefill_128k"], world, rank, args.shard)
             sp_steps = max(3, args.steps // 10)  # ~11 ms per step
             stimes, pairs = bench_prefill_sparse(ws_, dev, sp_steps, min(args.warmup, 5), flush, stream)
             sms = max_over_ranks(sum(stimes) / len(stimes), world)
@@ -380,12 +391,15 @@ def run_ours(args):
         line = {
             "metric": "attention TFLOPS (causal GQA prefill, Llama-3-8B shape)" if w.causal else "attention TFLOPS",
             "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "strong" if (args.shard == "heads" and world > 1) else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
                        "dv": w.dv, "causal": w.causal, "flops_per_step_per_gpu": flops,
                        "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"},
+                       "parallelism": ("single GPU" if world == 1 else
+                                       f"head-sharded x{world} ({w.Hq} query heads per GPU)" if args.shard == "heads"
+                                       else f"independent replicas x{world}")},
             "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(per_gpu_tflops / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "algorithmic_flops_per_launch": flops, "traffic": None},
@@ -444,6 +458,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-f16", action="store_true", help="skip the fp16-input measurements")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse prefill measurement")
+    ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
+                    help="N > 1: each rank runs its own batch (weak scaling) or a head shard of one layer "
+                         "(strong scaling, no collective)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -61,3 +61,81 @@ def test_reference_arm_only_rank0_prints(capsys, monkeypatch):
         cpu_seconds = 0.1
     bench.run_reference(A())
     assert capsys.readouterr().out == ""
+
+
+# ------------------------------------------------------------------------------------------------
+# head sharding (tensor parallel over heads, no collective on the data path)
+# ------------------------------------------------------------------------------------------------
+def test_head_shard_rules():
+    from exact_attention_139_b200.shard import head_shard
+    # Llama-3-8B shape over 4 ranks: whole groups of 4 query heads and their kv heads
+    s = [head_shard(32, 8, 4, r) for r in range(4)]
+    assert [x.q_heads for x in s] == [(0, 8), (8, 16), (16, 24), (24, 32)]
+    assert [x.kv_heads for x in s] == [(0, 2), (2, 4), (4, 6), (6, 8)]
+    # MLA: 128 query heads on one latent head over 8 GPUs, 16 heads each, latent head replicated
+    s = [head_shard(128, 1, 8, r) for r in range(8)]
+    assert all(x.Hq == 16 and x.kv_heads == (0, 1) for x in s)
+    # a group of 8 spread over 2 ranks of 4 heads: each holds a copy of its kv head
+    assert head_shard(16, 2, 4, 3).kv_heads == (1, 2)
+    # uneven heads, groups of 6 cut into 4s, rank out of range, Hq not a multiple of Hkv
+    for bad in [(32, 8, 3, 0), (24, 4, 6, 0), (32, 8, 4, 4), (30, 4, 2, 0)]:
+        with pytest.raises(ValueError):
+            head_shard(*bad)
+
+
+def _shard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import numpy as np
+    from exact_attention_139_b200.inputs import Workload, make_inputs
+    from exact_attention_139_b200.shard import head_shard, shard_inputs
+    from oracle import oracle
+    results = {}
+    for name, w in [("gqa", Workload("sh", 2, 8, 2, 9, 13, 16, 16, True, seed=77)),
+                    ("mla", Workload("sh_mla", 2, 8, 1, 2, 21, 24, 16, True, latent=True, seed=78))]:
+        q, k, v = make_inputs(w)  # every rank draws the same global inputs
+        sh = head_shard(w.Hq, w.Hkv, world, rank)
+        qs, ks, vs = shard_inputs(q, k, v, sh)
+        o, lse = oracle.attn(qs, ks, vs, B=w.B, Hq=sh.Hq, Hkv=sh.Hkv, Lq=w.Lq, Lk=w.Lk, d=w.d, dv=w.dv,
+                             ldv=w.ldv, scale=w.scale, causal=w.causal)
+        results[name] = (o, lse)
+    out[rank] = results
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_head_shards_reassemble_the_layer():
+    """Each of two gloo ranks computes its head shard; the shards, gathered in rank order, equal
+    the unsharded layer (heads are independent: no exchange is needed)."""
+    import numpy as np
+    from exact_attention_139_b200.inputs import Workload, make_inputs
+    from oracle import oracle
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for name, w in [("gqa", Workload("sh", 2, 8, 2, 9, 13, 16, 16, True, seed=77)),
+                    ("mla", Workload("sh_mla", 2, 8, 1, 2, 21, 24, 16, True, latent=True, seed=78))]:
+        q, k, v = make_inputs(w)
+        o, lse = oracle.attn(q, k, v, B=w.B, Hq=w.Hq, Hkv=w.Hkv, Lq=w.Lq, Lk=w.Lk, d=w.d, dv=w.dv, ldv=w.ldv,
+                             scale=w.scale, causal=w.causal)
+        og = np.concatenate([res[r][name][0] for r in range(world)], axis=1)
+        lg = np.concatenate([res[r][name][1] for r in range(world)], axis=1)
+        assert np.array_equal(og, o) and np.array_equal(lg, lse)
+
+
+def test_bench_job_workload_modes():
+    import bench
+    from exact_attention_139_b200.inputs import WORKLOADS
+    w = WORKLOADS["llama8b_prefill_8k"]
+    b = bench.job_workload(w, 4, 1, "batch")
+    assert (b.Hq, b.Hkv, b.B) == (32, 8, 1) and b.seed != w.seed
+    h = bench.job_workload(w, 4, 1, "heads")
+    assert (h.Hq, h.Hkv, h.Lq) == (8, 2, 8192)
+    assert h.flops() * 4 == w.flops()  # the shards add up to the layer
+    m = bench.job_workload(WORKLOADS["mla_decode_64k"], 8, 7, "heads")
+    assert (m.Hq, m.Hkv, m.latent) == (2, 1, True) and m.kv_bytes() == WORKLOADS["mla_decode_64k"].kv_bytes()
+    assert bench.job_workload(w, 1, 0, "heads") == w
