@@ -230,26 +230,64 @@ def attn_selftest_wait_timeout(limit_us: int, device=None):
     _check(_lib.attn_selftest_wait_timeout(int(limit_us), _stream_handle(dev)), "attn_selftest_wait_timeout")
 
 
-def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
-                  device="cuda:0", bufs: dict | None = None):
-    """Host (CPU, ideally pinned) tensors in, host tensors out: copy in, attn_fwd, copy out.
+def _host_chunks(B: int, Hkv: int, want: int):
+    """(b, kv0, kv1) pieces of the [B, Hkv] unit grid, each inside one batch so that its q, k, v,
+    o and lse rows are contiguous in memory; about `want` pieces in total."""
+    per_b = max(1, -(-want // B))
+    step = max(1, -(-Hkv // per_b))
+    return [(b, k0, min(Hkv, k0 + step)) for b in range(B) for k0 in range(0, Hkv, step)]
 
-    ``bufs`` may hold reusable device / pinned buffers (keys q, k, v, o, lse, o_host, lse_host)."""
+
+def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
+                  device="cuda:0", bufs: dict | None = None, chunks: int = 4):
+    """Host (CPU, pinned) tensors in, host tensors out: copy in, attn_fwd, copy out, pipelined.
+
+    The (batch, kv head) grid is cut into about ``chunks`` contiguous pieces; piece i is copied
+    in on one stream, computed on a second and copied out on a third, so the host-to-device
+    copies, the kernels and the device-to-host copies of different pieces overlap. ``bufs`` may
+    hold the reusable device buffers, pinned outputs, streams and events between calls."""
     dev = torch.device(device)
     bufs = {} if bufs is None else bufs
     B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
     dv = v.shape[-1]
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if name not in bufs:
-            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
-        bufs[name].copy_(t, non_blocking=True)
+    G = Hq // Hkv
     if "o" not in bufs:
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
         bufs["o"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=dev)
         bufs["lse"] = torch.empty((B, Hq, Lq), dtype=torch.float32, device=dev)
         bufs["o_host"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, pin_memory=True)
         bufs["lse_host"] = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
-    attn_fwd(bufs["q"], bufs["k"], bufs["v"], causal=causal, scale=scale, out=bufs["o"], lse=bufs["lse"])
-    bufs["o_host"].copy_(bufs["o"], non_blocking=True)
-    bufs["lse_host"].copy_(bufs["lse"], non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
+        bufs["streams"] = [torch.cuda.Stream(dev) for _ in range(3)]
+    s_in, s_run, s_out = bufs["streams"]
+    main = torch.cuda.current_stream(dev)
+    s_in.wait_stream(main)  # earlier work on the caller's stream (e.g. a previous call) comes first
+    dq, dk, dvv, do, dl = bufs["q"], bufs["k"], bufs["v"], bufs["o"], bufs["lse"]
+    pieces = _host_chunks(B, Hkv, chunks)
+    done_out = []
+    for b, k0, k1 in pieces:
+        h0, h1 = k0 * G, k1 * G
+        e_in = torch.cuda.Event()
+        with torch.cuda.stream(s_in):
+            dq[b, h0:h1].copy_(q[b, h0:h1], non_blocking=True)
+            dk[b, k0:k1].copy_(k[b, k0:k1], non_blocking=True)
+            dvv[b, k0:k1].copy_(v[b, k0:k1], non_blocking=True)
+            e_in.record(s_in)
+        e_run = torch.cuda.Event()
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(e_in)
+            attn_fwd(dq[b:b + 1, h0:h1], dk[b:b + 1, k0:k1], dvv[b:b + 1, k0:k1], causal=causal, scale=scale,
+                     out=do[b:b + 1, h0:h1], lse=dl[b:b + 1, h0:h1])
+            e_run.record(s_run)
+        e_out = torch.cuda.Event()
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e_run)
+            bufs["o_host"][b, h0:h1].copy_(do[b, h0:h1], non_blocking=True)
+            bufs["lse_host"][b, h0:h1].copy_(dl[b, h0:h1], non_blocking=True)
+            e_out.record(s_out)
+        done_out.append(e_out)
+    for e in done_out:
+        main.wait_event(e)
+    main.synchronize()
     return bufs["o_host"], bufs["lse_host"]
