@@ -263,12 +263,14 @@ def bench_decode(w, dev, steps, warmup, flush, stream):
     qd, kd = q.to(dev), k.to(dev)
     vd = kd if w.latent else v.to(dev)
     del q, k, v
+    # num_splits = 0: the library's own schedule (balanced over the SMs for the tensor-core kernel);
+    # `splits` reports its partial-slot count
     splits = attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv)
-    ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, splits),
+    ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, 0),
                      dtype=torch.uint8, device=dev)
     o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=w.torch_dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
-    step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=splits,
+    step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=0,
                                     workspace=ws, out=o, lse=lse)
     times = time_steps(step, steps, warmup, flush, stream)
     if attn.attn_check_device() != attn.ATTN_OK:

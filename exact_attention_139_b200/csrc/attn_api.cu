@@ -172,6 +172,45 @@ int decode_ctas_per_sm(int impl, bool dense_v, int d) {
   return (impl == ATTN_DECODE_TCGEN05_N && dense_v && d == 128) ? kDenseTn128Occupancy : 1;
 }
 
+// How a decode call cuts the keys. Split mode: `splits` equal chunks of every unit (grid
+// splits x units). Balanced mode (queries-on-M kernel, num_splits == 0): one CTA per slot of the
+// GPU, each taking bal_w consecutive keys of the flattened (unit, key) space, bal_w <= Lk so a
+// CTA touches at most two units; `splits` is then the most partials any unit gets.
+struct DecodePlan {
+  int splits;
+  int bal_w;
+  long long ctas;
+};
+
+DecodePlan balanced_plan(long long units, int Lk, int slots) {
+  DecodePlan d{0, 0, 0};
+  const long long total = units * Lk;
+  long long w = (total + slots - 1) / slots;
+  w = (w + 63) / 64 * 64;
+  if (w > Lk || w > 0x7fffffffLL) return d;  // a CTA would span more than two units
+  int most = 1;
+  for (long long u = 0; u < units; ++u) {
+    const long long pieces = ((u + 1) * Lk - 1) / w - (u * Lk) / w + 1;
+    most = (int)std::max<long long>(most, pieces);
+  }
+  if (most > 256) return d;
+  d.splits = most;
+  d.bal_w = (int)w;
+  d.ctas = (total + w - 1) / w;
+  return d;
+}
+
+DecodePlan plan_decode(int impl, bool dense_v, int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int num_splits) {
+  if (num_splits > 0) return DecodePlan{num_splits, 0, 0};
+  const int sms = current_sm_count();
+  const int occ = decode_ctas_per_sm(impl, dense_v, d);
+  if (impl == ATTN_DECODE_TCGEN05_N) {
+    const DecodePlan bal = balanced_plan((long long)B * Hkv, Lk, sms * occ);
+    if (bal.bal_w > 0) return bal;
+  }
+  return DecodePlan{choose_splits(B, Hq, Hkv, Lq, Lk, dv, sms, occ), 0, 0};
+}
+
 template <int RMAX, int CPT, typename E>
 attn_status launch_cc(const DecodeParams& p, int splits, cudaStream_t st) {
   const size_t smem = attn::decode_cc_smem_bytes(p.R, p.d, p.dv, !p.v_is_k);
@@ -237,6 +276,7 @@ attn_status launch_tn(const DecodeParams& p, int splits, cudaStream_t st) {
   auto kern = attn::decode_tn_kernel<DCH, NPIECE, BK, NST, SEPV, E>;
   if (!allow_smem(kern, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(splits, p.B * p.Hkv);
+  if (p.bal_w > 0) grid = dim3((unsigned)((p.bal_total + p.bal_w - 1) / p.bal_w), 1);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tq, tkv, tv, p);
   return launch_status();
 }
@@ -286,10 +326,10 @@ attn_status launch_tc_any(const DecodeParams& p, int splits, cudaStream_t st) {
 
 template <typename E>
 attn_status launch_combine(const float* o_part, const float* lse_part, void* o, float* lse, long long rows, int dv,
-                           int splits, cudaStream_t st) {
+                           int splits, cudaStream_t st, int bal_w = 0, int Lk = 0, int R = 1) {
   if (rows <= 0) return ATTN_OK;
   attn::combine_kernel<E><<<(unsigned)rows, attn::kCombineThreads, 0, st>>>(
-      o_part, lse_part, reinterpret_cast<uint16_t*>(o), lse, rows, dv, splits);
+      o_part, lse_part, reinterpret_cast<uint16_t*>(o), lse, rows, dv, splits, bal_w, Lk, R);
   return launch_status();
 }
 
@@ -410,9 +450,8 @@ attn_status decode_impl(const void* q, const void* k, const void* v, void* o, fl
   if (impl == ATTN_DECODE_TCGEN05_N && !tn_ok) return ATTN_ERR_UNSUPPORTED;
   if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
   const bool dense_v = !(v == k && ldv == d);
-  int splits = num_splits;
-  if (splits == 0)
-    splits = choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), decode_ctas_per_sm(impl, dense_v, d));
+  const DecodePlan plan = plan_decode(impl, dense_v, B, Hq, Hkv, Lq, Lk, d, dv, num_splits);
+  const int splits = plan.splits;
   const long long rows = (long long)B * Hq * Lq;
   const size_t need = workspace_bytes(rows, dv, splits);
   if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return ATTN_ERR_WORKSPACE;
@@ -437,6 +476,8 @@ attn_status decode_impl(const void* q, const void* k, const void* v, void* o, fl
   p.causal = causal ? 1 : 0;
   p.chunk = split_chunk(Lk, splits);
   p.v_is_k = (v == k && ldv == d) ? 1 : 0;
+  p.bal_w = plan.bal_w;
+  p.bal_total = (long long)B * Hkv * Lk;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
@@ -451,7 +492,7 @@ attn_status decode_impl(const void* q, const void* k, const void* v, void* o, fl
     else st = cpt == 1 ? launch_cc<64, 1, E>(p, splits, cs) : launch_cc<64, 2, E>(p, splits, cs);
   }
   if (st != ATTN_OK) return st;
-  return launch_combine<E>(p.o_part, p.lse_part, o, lse, rows, dv, splits, cs);
+  return launch_combine<E>(p.o_part, p.lse_part, o, lse, rows, dv, splits, cs, p.bal_w, Lk, p.R);
 }
 
 }  // namespace
@@ -512,19 +553,22 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || dv < 1 || num_splits < 0 || num_splits > 256) return 0;
   if (Hq % Hkv != 0) return 0;
   if (num_splits > 0) return workspace_bytes((long long)B * Hq * Lq, dv, num_splits);
-  // enough for the count attn_decode chooses with either kernel occupancy
-  const int sms = current_sm_count();
-  const int s1 = choose_splits(B, Hq, Hkv, Lq, Lk, dv, sms, 1);
-  const int s2 = choose_splits(B, Hq, Hkv, Lq, Lk, dv, sms, kDenseTn128Occupancy);
-  return workspace_bytes((long long)B * Hq * Lq, dv, std::max(s1, s2));
+  // enough for whatever attn_decode plans for this shape: either kernel family, either occupancy
+  int most = 1;
+  for (int impl : {ATTN_DECODE_TCGEN05_N, ATTN_DECODE_CUDA_CORE})
+    for (bool dense : {false, true})
+      for (int dd : {128, 0})
+        most = std::max(most, plan_decode(impl, dense, B, Hq, Hkv, Lq, Lk, dd, dv, 0).splits);
+  return workspace_bytes((long long)B * Hq * Lq, dv, most);
 }
 
 int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
-  // dv == d == 128 is taken to be a dense V on the queries-on-M kernel (the GQA decode shape)
+  // the queries-on-M kernel serves R <= 32 rows per kv head; dv == d == 128 is taken to be a
+  // dense V (the GQA decode shape)
   const int R = (Hq / Hkv) * Lq;
-  const int occ = (dv == d && d == 128 && R <= 32) ? kDenseTn128Occupancy : 1;
-  return choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(), occ);
+  const int impl = R <= 32 ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
+  return plan_decode(impl, dv == d && d == 128, B, Hq, Hkv, Lq, Lk, d, dv, 0).splits;
 }
 
 attn_status attn_decode_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -592,16 +636,13 @@ attn_status attn_decode_noalloc(const void* q, const void* k, const void* v, voi
   if (st != ATTN_OK) return st;
   if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
   const int impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
-  const int splits =
-      num_splits > 0 ? num_splits
-                     : choose_splits(B, Hq, Hkv, Lq, Lk, dv, current_sm_count(),
-                                     decode_ctas_per_sm(impl, !(v == k && ldv == d), d));
-  const size_t need = workspace_bytes((long long)B * Hq * Lq, dv, splits);
+  const DecodePlan plan = plan_decode(impl, !(v == k && ldv == d), B, Hq, Hkv, Lq, Lk, d, dv, num_splits);
+  const size_t need = workspace_bytes((long long)B * Hq * Lq, dv, plan.splits);
   if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != ATTN_OK) return st;
-  return attn_decode_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, splits, scratch,
+  return attn_decode_ex(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits, scratch,
                         (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES, ATTN_DECODE_AUTO, stream);
 }
 

@@ -3,7 +3,9 @@
 // Chunks cover disjoint key ranges, so with per-chunk results (O_s normalised by its own sum,
 // lse_s = ln of its sum) the whole-row result is LSE = ln sum_s exp(lse_s) and
 // O = sum_s exp(lse_s - LSE) * O_s. A chunk with lse_s = -inf has no visible key and no weight.
-// One CTA per query row; threads stride over the dv columns, four at a time.
+// One CTA per query row; threads stride over the dv columns, four at a time. With the balanced
+// decode schedule (bal_w > 0) the number of partials differs per unit (R rows each): the CTAs
+// that cover keys u * Lk .. (u + 1) * Lk - 1, each bal_w keys wide, one partial apiece.
 #pragma once
 
 #include "sm100.cuh"
@@ -16,8 +18,12 @@ template <typename E>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    uint16_t* __restrict__ o, float* __restrict__ lse, long long rows, int dv,
-                   int num_splits) {
+                   int num_splits, int bal_w, int Lk, int R) {
   const long long row = blockIdx.x;
+  if (bal_w > 0) {
+    const long long u = row / R;
+    num_splits = (int)(((u + 1) * Lk - 1) / bal_w - (u * Lk) / bal_w + 1);
+  }
   float m = -INFINITY;
   for (int s = 0; s < num_splits; ++s) m = fmaxf(m, lse_part[(long long)s * rows + row]);
   float L = -INFINITY;

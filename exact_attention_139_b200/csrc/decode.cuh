@@ -32,7 +32,40 @@ struct DecodeParams {
   int chunk;  // keys per split (multiple of 64)
   int v_is_k;
   float scale_log2;
+  // Balanced schedule (queries-on-M kernel, bal_w > 0): CTA c takes keys [c * bal_w, (c + 1) *
+  // bal_w) of the flattened (unit, key) space, unit = batch * Hkv + kv head, bal_total = units * Lk
+  // keys in all; bal_w <= Lk, so a CTA covers at most two units. Its part of unit u goes to
+  // partial slot c - first_cta(u), first_cta(u) = (u * Lk) / bal_w.
+  int bal_w;
+  long long bal_total;
 };
+
+// One contiguous key range of one unit processed by a CTA, and the partial slot it fills.
+struct DecodeSeg {
+  int unit, j_begin, j_end, piece;
+};
+
+// The segments of this CTA: one (split mode: split blockIdx.x of unit blockIdx.y, possibly
+// empty) or up to two (balanced mode).
+__device__ __forceinline__ int decode_segments(const DecodeParams& p, DecodeSeg (&seg)[2]) {
+  if (p.bal_w == 0) {
+    const int jb = blockIdx.x * p.chunk;
+    seg[0] = DecodeSeg{(int)blockIdx.y, jb, min(p.Lk, jb + p.chunk), (int)blockIdx.x};
+    return 1;
+  }
+  const long long pos0 = (long long)blockIdx.x * p.bal_w;
+  const long long pos1 = min(p.bal_total, pos0 + p.bal_w);
+  int n = 0;
+  for (long long pos = pos0; pos < pos1 && n < 2;) {
+    const int u = (int)(pos / p.Lk);
+    const long long ub = (long long)u * p.Lk;
+    const int jb = (int)(pos - ub);
+    const int je = (int)min((long long)p.Lk, pos1 - ub);
+    seg[n++] = DecodeSeg{u, jb, je, (int)(blockIdx.x - ub / p.bal_w)};
+    pos = ub + je;
+  }
+  return n;
+}
 
 // ======================================================================================
 // CUDA-core kernel
@@ -588,8 +621,8 @@ struct DecodeTnCfg {
   static constexpr int OFF_PAD = OFF_P + 2 * PB;    // 4 KB of slack read as rows 32..63 of P1
   static constexpr int OFF_BAR = OFF_PAD + 4096;
   // barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_full[2], pv_done[2],
-  // drain[1 + NACC] (one per MMA-issuing warp)
-  static constexpr int N_BARS = 1 + 2 * NST + 6 + 1 + NACC;
+  // drain[1 + NACC] (one per MMA-issuing warp), q_empty, o_free
+  static constexpr int N_BARS = 1 + 2 * NST + 6 + 1 + NACC + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
   static constexpr uint32_t S_COL = 0;
@@ -641,13 +674,15 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
   uint8_t* smem = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int split = blockIdx.x;
-  const int unit = blockIdx.y;
-  const int b = unit / p.Hkv, hkv = unit % p.Hkv;
-  const long long row0 = ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
-  const int j_begin = split * p.chunk;
-  const int j_end = min(p.Lk, j_begin + p.chunk);
-  const int n_tiles = j_end > j_begin ? (j_end - j_begin + BK - 1) / BK : 0;
+  DecodeSeg seg[2];
+  const int nseg = decode_segments(p, seg);
+  auto seg_tiles = [&](int g) {
+    return seg[g].j_end > seg[g].j_begin ? (seg[g].j_end - seg[g].j_begin + BK - 1) / BK : 0;
+  };
+  auto seg_row0 = [&](int g) {
+    const int b = seg[g].unit / p.Hkv, hkv = seg[g].unit % p.Hkv;
+    return ((long long)b * p.Hq + (long long)hkv * p.G) * p.Lq;
+  };
   const int off = p.Lk - p.Lq;
   const int NW = p.dv / NPIECE;  // columns per O piece (multiple of 64)
   // TMEM columns: O needs dv (lane half 0), the S partial tiles 2 * NACC * BK (lane half 1)
@@ -661,6 +696,8 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
   const uint32_t bar_p_full = bar_s_full + 16;
   const uint32_t bar_pv_done = bar_p_full + 16;
   const uint32_t bar_drain = bar_pv_done + 16;
+  const uint32_t bar_q_empty = bar_drain + 8 * (1 + C::NACC);  // all S of a segment issued and done
+  const uint32_t bar_o_free = bar_q_empty + 8;                 // the softmax has read O out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
 
   if (threadIdx.x == 0) {
@@ -675,6 +712,8 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
       mbar_init(bar_pv_done + 8 * i, 1);
     }
     for (int i = 0; i <= C::NACC; ++i) mbar_init(bar_drain + 8 * i, 1);
+    mbar_init(bar_q_empty, C::NACC);
+    mbar_init(bar_o_free, 64);
     fence_mbar_init();
   }
   if (warp == 3) {
@@ -688,65 +727,83 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
 
   if (warp == 2) {
     // ------------------------------- TMA producer -------------------------------
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kv);
       if constexpr (SEPV) tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q, DCH * C::QCH);
-#pragma unroll
-      for (int c = 0; c < DCH; ++c) tma_load_2d(base + C::OFF_Q + c * C::QCH, &tm_q, bar_q, 64 * c, (int)row0);
-      const int z = b * p.Hkv + hkv;
-      int t = 0;
+      int t = 0, qn = 0;  // tiles and Q tiles loaded so far
       bool ok = true;
-      for (; t < n_tiles; ++t) {
-        const int s = t % NST;
-        if (t >= NST) ok = mbar_wait(bar_kv_empty + 8 * s, ((t / NST) & 1) ^ 1, 41);
+      for (int g = 0; g < nseg && ok; ++g) {
+        const int n_tiles = seg_tiles(g);
+        if (n_tiles == 0) continue;
+        // Q of this segment's unit, once every S product of the previous segment is done
+        if (qn > 0) ok = mbar_wait(bar_q_empty, (qn - 1) & 1, 40);
         if (!ok) break;
-        const uint32_t full = bar_kv_full + 8 * s;
-        mbar_arrive_expect_tx(full, C::STAGE);
+        mbar_arrive_expect_tx(bar_q, DCH * C::QCH);
 #pragma unroll
-        for (int c = 0; c < DCH; ++c)
-          tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j_begin + t * BK, z);
-        if constexpr (SEPV) {
+        for (int c = 0; c < DCH; ++c) tma_load_2d(base + C::OFF_Q + c * C::QCH, &tm_q, bar_q, 64 * c, (int)seg_row0(g));
+        ++qn;
+        const int z = seg[g].unit;
+        for (int tt = 0; tt < n_tiles; ++tt, ++t) {
+          const int s = t % NST;
+          if (t >= NST) ok = mbar_wait(bar_kv_empty + 8 * s, ((t / NST) & 1) ^ 1, 41);
+          if (!ok) break;
+          const uint32_t full = bar_kv_full + 8 * s;
+          const int j = seg[g].j_begin + tt * BK;
+          mbar_arrive_expect_tx(full, C::STAGE);
 #pragma unroll
           for (int c = 0; c < DCH; ++c)
-            tma_load_3d(base + C::OFF_KV + s * C::STAGE + C::VOFF + c * C::KCH, &tm_v, full, 64 * c, j_begin + t * BK, z);
+            tma_load_3d(base + C::OFF_KV + s * C::STAGE + c * C::KCH, &tm_kv, full, 64 * c, j, z);
+          if constexpr (SEPV) {
+#pragma unroll
+            for (int c = 0; c < DCH; ++c)
+              tma_load_3d(base + C::OFF_KV + s * C::STAGE + C::VOFF + c * C::KCH, &tm_v, full, 64 * c, j, z);
+          }
         }
       }
       if (!ok) {
-        mbar_wait_drain(bar_q, 0);
+        if (qn > 0) mbar_wait_drain(bar_q, (qn - 1) & 1);
         for (int u = max(0, t - NST); u < t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u % NST), (u / NST) & 1);
       }
     }
   } else if (warp >= 4) {
     // -------------------- S issuers: partial a = chunks a, a + NACC, ... --------------------
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(64, BK, false, false, E::kFmt);  // S = Q.K^T
       const int a = warp - 4;
       const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL + a * BK;
       const uint64_t qdesc = make_sdesc(base + C::OFF_Q + a * C::QCH, 16, 1024, kSwizzle128B);
-      bool ok = mbar_wait(bar_q, 0, 42);
-      bool issued = false;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
-        // S buffer (t & 1) was last read by the softmax of tile t - 2
-        if (ok && t >= 2) ok = mbar_wait(bar_p_full + 8 * (t & 1), ((t - 2) >> 1) & 1, 50);
+      bool ok = true, issued = false;
+      int t = 0, qn = 0;
+      for (int g = 0; g < nseg && ok; ++g) {
+        const int n_tiles = seg_tiles(g);
+        if (n_tiles == 0) continue;
+        ok = mbar_wait(bar_q, qn & 1, 42);
         if (!ok) break;
-        tc_fence_after();
-        const uint64_t kdesc = make_sdesc(base + C::OFF_KV + (t % NST) * C::STAGE + a * C::KCH, 16, 1024, kSwizzle128B);
-        const uint32_t d = s_tmem + (t & 1) * C::NACC * BK;
+        ++qn;
+        for (int tt = 0; tt < n_tiles && ok; ++tt, ++t) {
+          ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
+          // S buffer (t & 1) was last read by the softmax of tile t - 2
+          if (ok && t >= 2) ok = mbar_wait(bar_p_full + 8 * (t & 1), ((t - 2) >> 1) & 1, 50);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t kdesc = make_sdesc(base + C::OFF_KV + (t % NST) * C::STAGE + a * C::KCH, 16, 1024, kSwizzle128B);
+          const uint32_t d = s_tmem + (t & 1) * C::NACC * BK;
 #pragma unroll
-        for (int i = 0; i < DCH / C::NACC; ++i) {
+          for (int i = 0; i < DCH / C::NACC; ++i) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            // descriptor start addresses advance by whole 16-byte units
-            const uint64_t qa = qdesc + (uint64_t)((i * C::NACC * C::QCH + ks * 32) >> 4);
-            const uint64_t kb = kdesc + (uint64_t)((i * C::NACC * C::KCH + ks * 32) >> 4);
-            mma_ss(d, qa, kb, idesc_s, (i > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {
+              // descriptor start addresses advance by whole 16-byte units
+              const uint64_t qa = qdesc + (uint64_t)((i * C::NACC * C::QCH + ks * 32) >> 4);
+              const uint64_t kb = kdesc + (uint64_t)((i * C::NACC * C::KCH + ks * 32) >> 4);
+              mma_ss(d, qa, kb, idesc_s, (i > 0 || ks > 0) ? 1u : 0u);
+            }
           }
+          issued = true;
+          mma_commit(bar_s_full + 8 * (t & 1));
         }
-        issued = true;
-        mma_commit(bar_s_full + 8 * (t & 1));
+        if (!ok) break;
+        mma_commit(bar_q_empty);  // this segment's Q may be replaced once these products are done
       }
       if (!ok && issued) {
         mma_commit(bar_drain + 8 * (1 + a));
@@ -755,30 +812,39 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
     }
   } else if (warp == 3) {
     // ------------------------------- P.V issuer -------------------------------
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       const uint32_t idesc_o = make_idesc(64, NW, false, true, E::kFmt);  // O += P.V
       bool ok = true, issued = false;
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
+      int t = 0, segs_done = 0;
+      for (int g = 0; g < nseg && ok; ++g) {
+        const int n_tiles = seg_tiles(g);
+        if (n_tiles == 0) continue;
+        // the first product of a segment overwrites O: the previous segment's O must be read out
+        if (segs_done > 0) ok = mbar_wait(bar_o_free, (segs_done - 1) & 1, 39);
         if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE + (SEPV ? C::VOFF : 0);  // V rows
-        const uint32_t pb = base + C::OFF_P + (t & 1) * C::PB;
+        for (int tt = 0; tt < n_tiles && ok; ++tt, ++t) {
+          ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE + (SEPV ? C::VOFF : 0);  // V rows
+          const uint32_t pb = base + C::OFF_P + (t & 1) * C::PB;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
 #pragma unroll
-          for (int h = 0; h < NPIECE; ++h) {
-            // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
-            const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
-            mma_ss(tmem + h * NW, ad, bd, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
+            for (int h = 0; h < NPIECE; ++h) {
+              // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
+              const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
+              mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          issued = true;
+          // the S products of this tile completed before its softmax started, so this commit
+          // also covers every read of the stage
+          mma_commit(bar_kv_empty + 8 * (t % NST));
+          mma_commit(bar_pv_done + 8 * (t & 1));
         }
-        issued = true;
-        // the S products of this tile completed before its softmax started, so this commit
-        // also covers every read of the stage
-        mma_commit(bar_kv_empty + 8 * (t % NST));
-        mma_commit(bar_pv_done + 8 * (t & 1));
+        ++segs_done;
       }
       if (!ok && issued) {
         mma_commit(bar_drain);
@@ -793,105 +859,112 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
     const int qi = m % p.Lq;
     const uint32_t tw = tmem + ((uint32_t)(warp * 32) << 16);
     const float c2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int t = 0; t < n_tiles; ++t) {
-      ok = mbar_wait(bar_s_full + 8 * (t & 1), (t >> 1) & 1, 45);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float x[64];
-      tmem_ld_keys<BK>(tw + C::S_COL + (t & 1) * C::NACC * BK, x);
-#pragma unroll
-      for (int a = 1; a < C::NACC; ++a) {
-        float y[64];
-        tmem_ld_keys<BK>(tw + C::S_COL + ((t & 1) * C::NACC + a) * BK, y);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < BK; ++e) x[e] += y[e];
-      }
-      tmem_wait_ld();
-      const int k0 = j_begin + t * BK;
-      int lim = j_end - 1;
-      if (p.causal) lim = min(lim, qi + off);
-      const int rem = lim - k0;  // keys c <= rem of this tile are visible
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < BK; ++e) {
-        if (e > rem) x[e] = -INFINITY;
-        mx = fmaxf(mx, x[e]);
-      }
-      const float m_tile = mx * c2;
-      float alpha = 1.f;
-      if (m_tile != -INFINITY) {
-        if (m_run == -INFINITY) {
-          m_run = m_tile;  // O row and l are still zero: nothing to rescale
-        } else if (m_tile > m_run + kRescaleLog2) {
-          alpha = ex2_approx(m_run - m_tile);
-          m_run = m_tile;
-        }
-      }
-      const float m_ref = (m_run == -INFINITY) ? 0.f : m_run;
-      // P buffer (t & 1) is free once P.V of tile t-2 has completed
-      if (t >= 2) {
-        ok = mbar_wait(bar_pv_done + 8 * (t & 1), ((t - 2) >> 1) & 1, 46);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-      }
-      float sum = 0.f;
-      uint8_t* prow = smem + C::OFF_P + (t & 1) * C::PB;
-#pragma unroll
-      for (int u = 0; u < BK / 8; ++u) {  // 8 keys per 16-byte unit
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(x[8 * u + 2 * e], c2, -m_ref));
-          const float p1 = ex2_approx(fmaf(x[8 * u + 2 * e + 1], c2, -m_ref));
-          sum += p0 + p1;
-          w4[e] = E::pack2(p0, p1);
-        }
-        if (s_lane)
-          *reinterpret_cast<uint4*>(prow + swz128_offset((uint32_t)m, (uint32_t)u)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      l_run = l_run * alpha + sum;
-      // rescale the O rows whose reference moved (rare): lanes 0-15 own those O rows
-      const float alpha_o = __shfl_down_sync(0xffffffffu, alpha, 16);
-      const bool need = t > 0 && __any_sync(0xffffffffu, s_lane && alpha != 1.f);
-      if (need) {
-        // O is stable once P.V of tile t-1 is done; S of tile t+1 (same columns, other lane
-        // half, rewritten unchanged below) must have landed too
-        ok = mbar_wait(bar_pv_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, 47);
-        if (ok && t + 1 < n_tiles) ok = mbar_wait(bar_s_full + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, 48);
+    int t = 0;
+    for (int g = 0; g < nseg && ok; ++g) {
+      const int n_tiles = seg_tiles(g);
+      const int j_begin = seg[g].j_begin, j_end = seg[g].j_end;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int tt = 0; tt < n_tiles; ++tt, ++t) {
+        ok = mbar_wait(bar_s_full + 8 * (t & 1), (t >> 1) & 1, 45);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const float a = s_lane ? 1.f : alpha_o;
-        for (int cg = 0; cg < p.dv / 32; ++cg) {
-          float o[32];
-          tmem_ld32(tw + 32 * cg, o);
+        float x[64];
+        tmem_ld_keys<BK>(tw + C::S_COL + (t & 1) * C::NACC * BK, x);
+#pragma unroll
+        for (int a = 1; a < C::NACC; ++a) {
+          float y[64];
+          tmem_ld_keys<BK>(tw + C::S_COL + ((t & 1) * C::NACC + a) * BK, y);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= a;
-          tmem_st32(tw + 32 * cg, o);
+          for (int e = 0; e < BK; ++e) x[e] += y[e];
         }
-        tmem_wait_st();
+        tmem_wait_ld();
+        const int k0 = j_begin + tt * BK;
+        int lim = j_end - 1;
+        if (p.causal) lim = min(lim, qi + off);
+        const int rem = lim - k0;  // keys c <= rem of this tile are visible
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < BK; ++e) {
+          if (e > rem) x[e] = -INFINITY;
+          mx = fmaxf(mx, x[e]);
+        }
+        const float m_tile = mx * c2;
+        float alpha = 1.f;
+        if (m_tile != -INFINITY) {
+          if (m_run == -INFINITY) {
+            m_run = m_tile;  // O row and l are still zero: nothing to rescale
+          } else if (m_tile > m_run + kRescaleLog2) {
+            alpha = ex2_approx(m_run - m_tile);
+            m_run = m_tile;
+          }
+        }
+        const float m_ref = (m_run == -INFINITY) ? 0.f : m_run;
+        // P buffer (t & 1) is free once P.V of tile t-2 has completed
+        if (t >= 2) {
+          ok = mbar_wait(bar_pv_done + 8 * (t & 1), ((t - 2) >> 1) & 1, 46);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        float sum = 0.f;
+        uint8_t* prow = smem + C::OFF_P + (t & 1) * C::PB;
+#pragma unroll
+        for (int u = 0; u < BK / 8; ++u) {  // 8 keys per 16-byte unit
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2_approx(fmaf(x[8 * u + 2 * e], c2, -m_ref));
+            const float p1 = ex2_approx(fmaf(x[8 * u + 2 * e + 1], c2, -m_ref));
+            sum += p0 + p1;
+            w4[e] = E::pack2(p0, p1);
+          }
+          if (s_lane)
+            *reinterpret_cast<uint4*>(prow + swz128_offset((uint32_t)m, (uint32_t)u)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        l_run = l_run * alpha + sum;
+        // rescale the O rows whose reference moved (rare): lanes 0-15 own those O rows
+        const float alpha_o = __shfl_down_sync(0xffffffffu, alpha, 16);
+        const bool need = tt > 0 && __any_sync(0xffffffffu, s_lane && alpha != 1.f);
+        if (need) {
+          // O is stable once P.V of tile t-1 is done; S of tile t+1 (same columns, other lane
+          // half, rewritten unchanged below) must have landed too, whichever segment it is in
+          const bool next_tile = tt + 1 < n_tiles || (g + 1 < nseg && seg_tiles(g + 1) > 0);
+          ok = mbar_wait(bar_pv_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, 47);
+          if (ok && next_tile) ok = mbar_wait(bar_s_full + 8 * ((t + 1) & 1), ((t + 1) >> 1) & 1, 48);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const float sc = s_lane ? 1.f : alpha_o;
+          for (int cg = 0; cg < p.dv / 32; ++cg) {
+            float o[32];
+            tmem_ld32(tw + 32 * cg, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= sc;
+            tmem_st32(tw + 32 * cg, o);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_p_full + 8 * (t & 1));
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_p_full + 8 * (t & 1));
-    }
-    if (ok && n_tiles > 0) {
-      ok = mbar_wait(bar_pv_done + 8 * ((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, 49);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) break;
+      if (n_tiles > 0) {
+        ok = mbar_wait(bar_pv_done + 8 * ((t - 1) & 1), ((t - 1) >> 1) & 1, 49);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
       // lanes 16-31 hold (m_run, l_run) of row m; lanes 0-15 hold O row m
+      const long long row0 = seg_row0(g);
+      const int piece = seg[g].piece;
       const float l_o = __shfl_down_sync(0xffffffffu, l_run, 16);
       if (s_lane && row_ok)
-        p.lse_part[(long long)split * p.rows_total + row0 + m] =
-            (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        p.lse_part[(long long)piece * p.rows_total + row0 + m] = (l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
       const float inv = (l_o > 0.f) ? 1.f / l_o : 0.f;
-      float* dst = p.o_part + ((long long)split * p.rows_total + row0 + m) * p.dv;
+      float* dst = p.o_part + ((long long)piece * p.rows_total + row0 + m) * p.dv;
       tc_fence_after();
       for (int cg = 0; cg < p.dv / 32; ++cg) {
         float o[32];
@@ -908,6 +981,9 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
             *reinterpret_cast<float4*>(dst + 32 * cg + e) = make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
         }
       }
+      // O may now be overwritten by the next segment's first P.V product
+      tc_fence_before();
+      mbar_arrive(bar_o_free);
     }
   }
 

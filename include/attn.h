@@ -140,7 +140,13 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv
  *
  *   v, ldv   V rows with stride ldv >= dv. MLA latent KV passes v == k and ldv == d: V is the
  *            first dv columns of each latent K row, and every row is read from memory once.
- *   num_splits  0 = chosen from the shape and the SM count; otherwise 1..256.
+ *   num_splits  1..256: every (batch, kv head) is cut into that many equal chunks. 0: the library's
+ *               schedule. For the queries-on-M kernel that is a balanced grid of one CTA per SM
+ *               slot, each taking an equal run of consecutive keys of the (batch * Hkv + kv head,
+ *               key) sequence (a run may end in one kv head and continue in the next), so every SM
+ *               streams the same number of bytes; a kv head then gets up to
+ *               attn_decode_default_splits(...) partials. Other kernels use equal chunks with a
+ *               count chosen from the shape and the SM count.
  *   workspace   device buffer of at least attn_decode_workspace_size(...) bytes, 256-byte
  *               aligned. Its contents on entry do not matter.
  * Supported: rows per kv head R = (Hq/Hkv)*Lq <= 64; d <= 576, dv <= 512, d and dv
@@ -221,7 +227,10 @@ attn_status attn_combine_typed(const float *o_part, const float *lse_part, void 
                                int B, int Hq, int Lq, int dv, int num_splits, int dtype,
                                void *stream);
 
-/* Number of splits attn_decode would choose (num_splits = 0) on the current device. */
+/* Number of partial results per (batch, kv head) that attn_decode uses with num_splits = 0 on the
+ * current device (the most any kv head gets under the balanced schedule). The shape is taken
+ * to have a dense V when dv == d == 128, latent KV otherwise; attn_decode_workspace_size with
+ * num_splits = 0 covers every case. */
 int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv);
 
 /*

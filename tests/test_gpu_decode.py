@@ -60,7 +60,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("splits", [1, 3, 16])
+@pytest.mark.parametrize("splits", [0, 1, 3, 16])  # 0: the library's schedule (balanced for TN)
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B{}_H{}x{}_Lq{}_Lk{}_d{}_{}".format(*s[:7]))
 def test_small_shapes(shape, splits, cuda_device):
     from exact_attention_139_b200 import attn
@@ -87,7 +87,7 @@ def test_split_count_invariance(cuda_device):
     from exact_attention_139_b200 import attn
     w = Workload("inv", 2, 16, 1, 2, 5000, 576, 512, True, latent=True, seed=31)
     q, k, _ = (t.to(cuda_device) for t in make_inputs(w))
-    outs = [attn.attn_decode(q, k, k, causal=True, dv=512, num_splits=s)[0].float() for s in (1, 5, 40)]
+    outs = [attn.attn_decode(q, k, k, causal=True, dv=512, num_splits=s)[0].float() for s in (1, 5, 40, 0)]
     for o in outs[1:]:
         assert (o - outs[0]).abs().max().item() <= 1e-2
 
@@ -121,3 +121,18 @@ def test_combine_against_oracle_merge(cuda_device):
     o2, l2 = attn.attn_combine(torch.tensor(op_empty, dtype=torch.float32, device=cuda_device),
                                torch.tensor(lp_empty, dtype=torch.float32, device=cuda_device), B=1, Hq=1, Lq=1)
     assert torch.all(o2 == 0) and torch.isinf(l2).all() and (l2 < 0).all()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,latent", [(3, 16, 1, 2, 1000, True), (5, 16, 1, 2, 4097, True),
+                                                  (2, 32, 8, 1, 3001, False), (7, 8, 2, 2, 777, False)])
+def test_balanced_schedule_vs_oracle(B, Hq, Hkv, Lq, Lk, latent, cuda_device):
+    """num_splits = 0 on the queries-on-M kernel: CTAs take equal ranges of the flattened
+    (unit, key) space, so ranges straddle units and the last piece of a unit may hold only keys
+    that the causal mask hides from its first query row."""
+    from exact_attention_139_b200 import attn
+    d, dv = (576, 512) if latent else (128, 128)
+    w = Workload("bal", B, Hq, Hkv, Lq, Lk, d, dv, True, latent=latent, seed=2500 + Lk)
+    q, k, v, o, lse = run(w, cuda_device, impl=TN, num_splits=0)
+    rows = np.arange(B * Hq * Lq)
+    o_ref, l_ref = oracle_rows(w, q, k, v, rows)
+    compare(o.reshape(-1, dv), lse.reshape(-1), o_ref, l_ref, f"balanced B{B} Lk{Lk}")
