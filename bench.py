@@ -38,6 +38,14 @@ import torch  # noqa: E402
 from exact_attention_139_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+# DRAM bytes (read + write) per launch of the timed kernel, from one ncu capture of the current
+# kernels (dram__bytes.sum.per_second x gpu__time_duration.sum; see profiles/): reported as the
+# roofline "traffic". Re-measure whenever one of these kernels changes.
+NCU_TRAFFIC_BYTES = {
+    "llama8b_prefill_8k": 132.6e6,   # prefill2_kernel<128, bf16, dense>
+    "mla_decode_64k": 2427.1e6,      # decode_tn_kernel<9,2,48,3,latent,bf16>, balanced grid
+    "gqa_decode_32k": 2154.3e6,      # decode_tn_kernel<2,1,48,3,dense V,bf16>, balanced grid
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -332,7 +340,8 @@ def run_ours(args):
             "per_gpu_gbs": round(ggbs, 1), "ms_per_step": round(gms, 4), "num_splits": gsplits,
             "roofline": {"bound": "hbm", "achieved": round(ggbs, 1), "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": round(ggbs / float(peaks["hbm_gbs"]), 4),
-                         "algorithmic_bytes_per_launch": wg.kv_bytes()}}
+                         "algorithmic_bytes_per_launch": wg.kv_bytes(),
+                         "traffic": NCU_TRAFFIC_BYTES.get(wg.name) if wg.Hq == 32 else None}}
         launches += 2 * args.steps
         extras["decode"] = {
             "workload": wd.name, "metric": "KV-read HBM GB/s", "value": round(gbs * world, 1),
@@ -340,7 +349,8 @@ def run_ours(args):
             "kernels_per_step": 2,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": peak_src,
-                         "algorithmic_bytes_per_launch": wd.kv_bytes(), "traffic": None,
+                         "algorithmic_bytes_per_launch": wd.kv_bytes(),
+                         "traffic": NCU_TRAFFIC_BYTES.get(wd.name) if wd.Hq == 16 else None,
                          "note": "step = split kernel + combine kernel"},
             "tflops": round(wd.flops() / (dms * 1e-3) / 1e12, 1), "clocks": dclk}
         launches += 2 * args.steps
@@ -404,7 +414,8 @@ def run_ours(args):
                                        else f"independent replicas x{world}")},
             "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(per_gpu_tflops / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
-                         "algorithmic_flops_per_launch": flops, "traffic": None},
+                         "algorithmic_flops_per_launch": flops,
+                         "traffic": NCU_TRAFFIC_BYTES.get(w.name) if world == 1 or args.shard == "batch" else None},
             "e2e": e2e,
             "gpu_launches": args.steps,  # one prefill kernel per timed step of the headline leg
             "gpu_launches_all_legs": launches,
