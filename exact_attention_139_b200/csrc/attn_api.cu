@@ -126,9 +126,9 @@ int split_chunk(int Lk, int splits) {
   return (c + 63) / 64 * 64;
 }
 
-// Choose the split count. Model: CTAs run one per SM in waves; a CTA costs its key tiles plus a
-// fixed start-up/drain cost of about kFixedTiles tiles (barrier set-up, Q load, ring fill, partial
-// write), and every split adds partial-result traffic. Minimise
+// Choose the split count of the equal-chunk grid. Model: CTAs run ctas_per_sm per SM in waves; a
+// CTA costs its key tiles plus a fixed start-up/drain cost of about kFixedTiles tiles (barrier
+// set-up, Q load, ring fill, partial write), and every split adds partial-result traffic. Minimise
 //   waves * (tiles per split + kFixedTiles) * (1 + partial bytes / KV bytes).
 // (On B200: mla_decode_64k -> 9 splits at one CTA per SM, gqa_decode_32k -> 9 at two CTAs per
 // SM, both the measured best: 4 to 28 splits were timed.)

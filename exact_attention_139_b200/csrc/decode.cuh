@@ -1,17 +1,21 @@
 // decode.cuh -- split-KV decode attention (few query tokens, long KV cache) on sm_100a.
 //
-// Each CTA takes one (batch, kv head, key chunk) and computes, for the R = (Hq/Hkv)*Lq query
-// rows that share the kv head, a partial O over its chunk (fp32, divided by its own softmax
-// sum) and the chunk's LSE (natural log; -inf when no key of the chunk is visible). The
-// log-sum-exp combine (combine.cuh) merges the chunks.
+// A CTA computes, for the R = (Hq/Hkv)*Lq query rows that share a kv head, a partial O over a
+// range of that head's keys (fp32, divided by its own softmax sum) and the range's LSE (natural
+// log; -inf when no key of the range is visible). The log-sum-exp combine (combine.cuh) merges
+// the partials. Ranges are equal chunks of every (batch, kv head) ("split mode"), or, for the
+// queries-on-M kernel with no split count given, equal runs of the flattened (batch * Hkv + kv
+// head, key) sequence with one CTA per SM slot ("balanced mode", DecodeParams::bal_w).
 //
-// Two kernels:
+// Three kernels:
 //   decode_cc_kernel      fp32 CUDA-core dot products; any supported shape; the baseline.
 //   decode_tc_kernel      tcgen05 with the key length on the MMA M dimension: the transposed
 //                         flow S^T = K.Q^T, P^T = softmax(S^T), O^T = V^T.P^T of the FlashMLA-ETAP
 //                         summary ("Mecanismo Central", items 1-3). With only R = 32 query rows
 //                         per kv head, putting keys (64 per tile) on M and queries on N avoids
 //                         padding the query dimension to the MMA's minimum M.
+//   decode_tn_kernel      tcgen05 with the query rows on M (padded to 64) and keys on N: every
+//                         softmax reduction stays inside one thread; the default.
 // Latent KV (MLA): V is the first dv columns of each K row; each row is read from HBM once and
 // the same shared-memory tile feeds both products. Dense V (GQA decode) streams beside K.
 #pragma once

@@ -15,13 +15,16 @@
 //         S_A(0) S_B(0) | PV_A(0) S_A(1) | PV_B(0) S_B(1) | PV_A(1) S_A(2) | ...
 //     A single issuing thread keeps each tile's products contiguous on the tensor core; issuing
 //     A and B from two warps interleaved them and was measured slower;
-//   * P (bf16) is written back into TMEM over the S columns it came from, and P.V takes its A
-//     operand from TMEM: shared memory holds only Q_A, Q_B and a 4-stage K/V ring, and the tensor
-//     core reads half as many operand bytes from shared memory as with P in shared memory (also
-//     measured: an SS-operand P.V made the kernel shared-memory-bandwidth bound);
-//   * the grid is persistent (one CTA per SM), units are handed out round-robin batch by batch in
-//     heaviest-first order (causal: last query tiles first), and every barrier phase carries
-//     across units.
+//   * P (16-bit) is written back into TMEM over the S columns it came from, and P.V takes its A
+//     operand from TMEM: shared memory holds only Q_A, Q_B and a K/V ring whose stage j holds
+//     K_j and V_j, and the tensor core reads half as many operand bytes from shared memory as
+//     with P in shared memory (also measured: an SS-operand P.V made the kernel
+//     shared-memory-bandwidth bound);
+//   * the grid is persistent (one CTA per SM); units are sorted by causal cost inside groups of
+//     batches whose K/V fits in half the L2 and dealt boustrophedon (see prefill_unit_index), and
+//     every barrier phase carries across units;
+//   * the block-sparse instantiation (SPARSE) walks the union of the two tiles' caller-given
+//     key-block lists instead of the causal prefix.
 // Warps: 0-7 softmax, 8 TMA producer, 9 TMEM allocator + MMA issuer.
 #pragma once
 
