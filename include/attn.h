@@ -53,7 +53,7 @@ extern "C" {
 typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_INVALID_ARG = 1, /* NULL pointer, non-positive size, Hq % Hkv, causal Lq > Lk */
-    ATTN_ERR_UNSUPPORTED = 2, /* valid attention, but a shape this build has no kernel for   */
+    ATTN_ERR_UNSUPPORTED = 2, /* valid attention, but a shape the library has no kernel for  */
     ATTN_ERR_MISALIGNED = 3,  /* a pointer or row stride breaks the 16-byte rule of TMA      */
     ATTN_ERR_WORKSPACE = 4,   /* decode workspace NULL or smaller than required             */
     ATTN_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed                        */
