@@ -440,14 +440,16 @@ def run_reference(args):
     for _ in range(args.warmup):
         oracle_sample_rate(w, min(2.0, args.cpu_seconds / 4), q, k, v)
     rows_used, threads = 0, 1
+    step_secs = []
     for _ in range(args.steps):
         rate, rows_used, secs, threads = oracle_sample_rate(w, args.cpu_seconds / max(1, args.steps), q, k, v)
         per_step.append(rate)
+        step_secs.append(secs)
     value = statistics.mean(per_step) / 1e12
     line = {
         "impl": "reference", "metric": "attention TFLOPS (causal GQA prefill, Llama-3-8B shape)",
         "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "ms_per_step": round(1e3 * statistics.mean(step_secs), 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16)",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
                    "dv": w.dv, "causal": w.causal},
