@@ -224,3 +224,34 @@ def test_sparse_argument_checks(lib):
     assert sp(cnt=0x60001) == MISALIGNED
     assert sp(d=96, dv=96) == UNSUPPORTED
     assert sp(q=A + 8) == MISALIGNED
+
+
+def _balanced_pieces(units, Lk, slots):
+    """Partials per kv head under the balanced schedule documented in attn.h / decode.cuh: runs of
+    W = ceil(units * Lk / slots) keys rounded up to 64 (None when W > Lk: equal chunks instead)."""
+    w = -(-units * Lk // slots)
+    w = -(-w // 64) * 64
+    if w > Lk:
+        return None
+    return max(((u + 1) * Lk - 1) // w - (u * Lk) // w + 1 for u in range(units))
+
+
+def test_decode_plan_balanced_schedule(lib):
+    """Without a GPU the library assumes 148 SMs; the latent kernel runs one CTA per SM, the dense
+    d = 128 kernel two."""
+    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 7
+    mla = lib.attn_decode_default_splits(32, 16, 1, 2, 65536, 576, 512)
+    assert mla == _balanced_pieces(32, 65536, 148)
+    gqa = lib.attn_decode_default_splits(16, 32, 8, 1, 32768, 128, 128)
+    assert gqa == _balanced_pieces(128, 32768, 296)
+    odd = lib.attn_decode_default_splits(3, 16, 1, 2, 4097, 576, 512)
+    assert odd == _balanced_pieces(3, 4097, 148)
+    # many short kv heads: a run would span more than two heads, so equal chunks are used
+    assert _balanced_pieces(64 * 8, 100, 296) is None
+    s = lib.attn_decode_default_splits(64, 32, 8, 1, 100, 128, 128)
+    assert 1 <= s <= 256
+    for (B, Hq, Hkv, Lq, Lk, d, dv), pieces in [((32, 16, 1, 2, 65536, 576, 512), mla),
+                                                 ((16, 32, 8, 1, 32768, 128, 128), gqa),
+                                                 ((3, 16, 1, 2, 4097, 576, 512), odd)]:
+        assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, 0) >= \
+            lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, pieces)
