@@ -255,3 +255,25 @@ def test_decode_plan_balanced_schedule(lib):
                                                  ((3, 16, 1, 2, 4097, 576, 512), odd)]:
         assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, 0) >= \
             lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, pieces)
+
+
+def _header_param_counts():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for name, params in re.findall(r"\b(attn_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = params.strip()
+        out[name] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_argtypes_match_header():
+    """Every function the Python binding declares has as many ctypes arguments as the C header."""
+    from exact_attention_139_b200 import attn
+    counts = _header_param_counts()
+    checked = 0
+    for name, n in counts.items():
+        fn = getattr(attn.lib(), name)
+        if getattr(fn, "argtypes", None) is not None:
+            assert len(fn.argtypes) == n, f"{name}: header {n} parameters, binding {len(fn.argtypes)}"
+            checked += 1
+    assert checked >= 10

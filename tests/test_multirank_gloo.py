@@ -139,3 +139,25 @@ def test_bench_job_workload_modes():
     m = bench.job_workload(WORKLOADS["mla_decode_64k"], 8, 7, "heads")
     assert (m.Hq, m.Hkv, m.latent) == (2, 1, True) and m.kv_bytes() == WORKLOADS["mla_decode_64k"].kv_bytes()
     assert bench.job_workload(w, 1, 0, "heads") == w
+
+
+def test_sparse_workload_index_structure():
+    """The sparse workload's given index: per query block a sorted, distinct list inside the causal
+    range that holds the first block, the diagonal block and the blocks of the biased keys."""
+    import numpy as np
+    from exact_attention_139_b200.inputs import Workload, block_lists, sparse_visible_pairs, vertical_positions
+    w = Workload("sp", 1, 4, 2, 2048, 2048, 16, 16, True, vertical_keys=8, vertical_bias=2.0, seed=5,
+                 sparse_window=3)
+    idx, cnt = block_lists(w)
+    pos = vertical_positions(w)
+    for h in range(w.Hq):
+        vb = set((pos[h // 2].numpy() // 128).tolist())
+        for qb in range(16):
+            lst = idx[0, h, qb, :cnt[0, h, qb]].tolist()
+            assert lst == sorted(set(lst)) and lst[0] == 0 and lst[-1] == qb
+            assert set(range(max(0, qb - 2), qb + 1)) <= set(lst)
+            assert {b for b in vb if b <= qb} <= set(lst)
+            assert all(b <= qb for b in lst)
+    full = sparse_visible_pairs(w, np.tile(np.arange(16, dtype=np.int32), (1, 4, 16, 1)),
+                                np.full((1, 4, 16), 16, dtype=np.int32))
+    assert full == w.visible_pairs()  # every block listed: the dense causal count
