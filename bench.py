@@ -337,7 +337,7 @@ def run_ours(args):
         ggbs = wg.kv_bytes() / (gms * 1e-3) / 1e9
         extras["decode_gqa"] = {
             "workload": wg.name, "metric": "KV-read HBM GB/s", "value": round(ggbs * world, 1),
-            "per_gpu_gbs": round(ggbs, 1), "ms_per_step": round(gms, 4), "num_splits": gsplits,
+            "per_gpu_gbs": round(ggbs, 1), "ms_per_step": round(gms, 4), "num_splits": gsplits, "schedule": "balanced grid (num_splits = most partials per kv head)",
             "roofline": {"bound": "hbm", "achieved": round(ggbs, 1), "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": round(ggbs / float(peaks["hbm_gbs"]), 4),
                          "algorithmic_bytes_per_launch": wg.kv_bytes(),
@@ -345,7 +345,7 @@ def run_ours(args):
         launches += 2 * args.steps
         extras["decode"] = {
             "workload": wd.name, "metric": "KV-read HBM GB/s", "value": round(gbs * world, 1),
-            "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits,
+            "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits, "schedule": "balanced grid (num_splits = most partials per kv head)",
             "kernels_per_step": 2,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": peak_src,
@@ -373,7 +373,7 @@ def run_ours(args):
             dfgbs = wdf.kv_bytes() / (dfms * 1e-3) / 1e9
             extras["decode_f16"] = {
                 "workload": wdf.name + " (fp16 inputs)", "metric": "KV-read HBM GB/s", "value": round(dfgbs * world, 1),
-                "ms_per_step": round(dfms, 4), "num_splits": dfsplits,
+                "ms_per_step": round(dfms, 4), "num_splits": dfsplits, "schedule": "balanced grid (num_splits = most partials per kv head)",
                 "roofline": {"bound": "hbm", "achieved": round(dfgbs, 1), "peak": float(peaks["hbm_gbs"]),
                              "unit": "GB/s", "frac": round(dfgbs / float(peaks["hbm_gbs"]), 4)}}
             launches += args.steps + 2 * args.steps
