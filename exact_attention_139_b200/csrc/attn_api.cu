@@ -328,8 +328,21 @@ template <typename E>
 attn_status launch_combine(const float* o_part, const float* lse_part, void* o, float* lse, long long rows, int dv,
                            int splits, cudaStream_t st, int bal_w = 0, int Lk = 0, int R = 1) {
   if (rows <= 0) return ATTN_OK;
-  attn::combine_kernel<E><<<(unsigned)rows, attn::kCombineThreads, 0, st>>>(
-      o_part, lse_part, reinterpret_cast<uint16_t*>(o), lse, rows, dv, splits, bal_w, Lk, R);
+  // programmatic dependent launch: the combine's CTAs may be scheduled while the previous kernel
+  // on the stream (the decode) drains; the kernel waits for that grid before reading partials
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(attn::kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn::combine_kernel<E>, o_part, lse_part, reinterpret_cast<uint16_t*>(o), lse, rows,
+                         dv, splits, bal_w, Lk, R) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   return launch_status();
 }
 

@@ -19,6 +19,9 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    uint16_t* __restrict__ o, float* __restrict__ lse, long long rows, int dv,
                    int num_splits, int bal_w, int Lk, int R) {
+  // launched as a programmatic dependent of the decode kernel: wait until that grid has finished
+  // and its partials are visible (returns at once for an ordinary launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long row = blockIdx.x;
   if (bal_w > 0) {
     const long long u = row / R;
