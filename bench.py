@@ -7,8 +7,9 @@ Llama-3-8B-shaped causal GQA prefill (B=1, Hq=32, Hkv=8, L=8192, d=128): metric 
 (algorithmic flops = 2*(d+dv) per visible query/key pair). The same JSON line also carries the
 MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) and the GQA
 decode (B=16, 32 query heads on 8 kv heads, Lk=32768) measured in HBM GB/s, and the fp16-input
-variants of the prefill and of the MLA decode, and the block-sparse 128K prefill over its given
-index, each with its roofline fraction against MEASURED_PEAKS.json.
+variants of the prefill and of the MLA decode, the 256-token batched prefill (against the larger
+of its compute and HBM times), and the 128K long-context prefill, dense and block-sparse over its
+given index, each with its roofline fraction against MEASURED_PEAKS.json.
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching stream;
 L2 is flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU (torchrun):
@@ -224,8 +225,10 @@ def bench_prefill(w, dev, steps, warmup, flush, stream):
     return times, (q, k, v)
 
 
-def bench_prefill_sparse(w, dev, steps, warmup, flush, stream):
-    """Block-sparse prefill over the workload's given index (inputs.block_lists)."""
+def bench_prefill_sparse(w, dev, steps, warmup, flush, stream, dense_steps=0):
+    """Block-sparse prefill over the workload's given index (inputs.block_lists); with dense_steps
+    > 0 also the dense causal prefill of the same inputs (the 128K long-context config: the sparse
+    workload shares its seeded Q, K, V)."""
     from exact_attention_139_b200 import attn
     from exact_attention_139_b200.inputs import block_lists, sparse_visible_pairs
     q, k, v = make_inputs(w)
@@ -238,9 +241,13 @@ def bench_prefill_sparse(w, dev, steps, warmup, flush, stream):
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
     step = lambda: attn.attn_fwd_sparse(qd, kd, vd, idx_d, cnt_d, causal=w.causal, scale=w.scale, out=o, lse=lse)
     times = time_steps(step, steps, warmup, flush, stream)
+    dense_times = []
+    if dense_steps > 0:
+        dstep = lambda: attn.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        dense_times = time_steps(dstep, dense_steps, 1, flush, stream)
     if attn.attn_check_device() != attn.ATTN_OK:
-        raise RuntimeError("device error during the sparse prefill benchmark")
-    return times, pairs
+        raise RuntimeError("device error during the 128K prefill benchmarks")
+    return times, pairs, dense_times
 
 
 def bench_prefill_e2e(w, dev, steps, warmup, host):
@@ -354,6 +361,20 @@ def run_ours(args):
                          "note": "step = split kernel + combine kernel"},
             "tflops": round(wd.flops() / (dms * 1e-3) / 1e12, 1), "clocks": dclk}
         launches += 2 * args.steps
+        # 256-token batched sweep: reported against the larger of its compute and HBM times (Q, K, V
+        # and O are 84 MB; the L2 is flushed before every step, so they come from HBM)
+        wsh = job_workload(WORKLOADS["batched_prefill_256"], world, rank, args.shard)
+        shtimes, _ = bench_prefill(wsh, dev, args.steps, args.warmup, flush, stream)
+        shms = max_over_ranks(sum(shtimes) / len(shtimes), world)
+        sh_bytes = 2 * (2 * wsh.B * wsh.Hq * wsh.Lq * wsh.d + wsh.B * wsh.Hkv * wsh.Lk * (wsh.d + wsh.dv))
+        t_bound = max(wsh.flops() / (peak_tf * 1e12), sh_bytes / (float(peaks["hbm_gbs"]) * 1e9))
+        extras["prefill_short"] = {
+            "workload": wsh.name, "metric": "attention TFLOPS", "value": round(wsh.flops() * world / (shms * 1e-3) / 1e12, 2),
+            "ms_per_step": round(shms, 4),
+            "roofline": {"bound": "max(tensor, hbm)", "achieved_ms": round(shms, 4), "bound_ms": round(t_bound * 1e3, 4),
+                         "frac": round(t_bound * 1e3 / shms, 4), "algorithmic_flops_per_launch": wsh.flops(),
+                         "algorithmic_bytes_per_launch": sh_bytes}}
+        launches += args.steps
         if not args.no_f16:
             # fp16 inputs: same kernels with the fp16 operand format; fp16 and bf16 share one
             # nominal tensor rate on B200, so the measured bf16 peak is the fp16 denominator
@@ -379,8 +400,10 @@ def run_ours(args):
             launches += args.steps + 2 * args.steps
         if not args.no_sparse:
             ws_ = job_workload(WORKLOADS["sparse_prefill_128k"], world, rank, args.shard)
-            sp_steps = max(3, args.steps // 10)  # ~11 ms per step
-            stimes, pairs = bench_prefill_sparse(ws_, dev, sp_steps, min(args.warmup, 5), flush, stream)
+            sp_steps = max(3, args.steps // 10)  # ~13 ms per step
+            long_steps = max(2, args.steps // 50)  # ~130 ms per step
+            stimes, pairs, ltimes = bench_prefill_sparse(ws_, dev, sp_steps, min(args.warmup, 5), flush, stream,
+                                                         dense_steps=long_steps)
             sms = max_over_ranks(sum(stimes) / len(stimes), world)
             sflops = pairs * 2.0 * (ws_.d + ws_.dv)
             stf = sflops / (sms * 1e-3) / 1e12
@@ -392,6 +415,15 @@ def run_ours(args):
                 "roofline": {"bound": "tensor", "achieved": round(stf, 2), "peak": peak_tf, "unit": "TFLOP/s",
                              "frac": round(stf / peak_tf, 4), "algorithmic_flops_per_launch": sflops}}
             launches += sp_steps
+            wl = job_workload(WORKLOADS["long_prefill_128k"], world, rank, args.shard)
+            lms = max_over_ranks(sum(ltimes) / len(ltimes), world)
+            ltf = wl.flops() / (lms * 1e-3) / 1e12
+            extras["prefill_long"] = {
+                "workload": wl.name, "metric": "attention TFLOPS", "value": round(ltf * world, 2),
+                "ms_per_step": round(lms, 3), "steps": long_steps,
+                "roofline": {"bound": "tensor", "achieved": round(ltf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                             "frac": round(ltf / peak_tf, 4), "algorithmic_flops_per_launch": wl.flops()}}
+            launches += long_steps
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
