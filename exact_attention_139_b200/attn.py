@@ -102,6 +102,51 @@ def _need(t: torch.Tensor, name: str, dtype=torch.bfloat16):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t: torch.Tensor, name: str, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _same_device(where: str, *ts):
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"{where}: tensors on different devices {sorted(map(str, devs))}")
+
+
+def _qkv_dims(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    """(B, Hq, Lq, d, Hkv, Lk, ldv) of q [B,Hq,Lq,d], k [B,Hkv,Lk,d], v [B,Hkv,Lk,ldv].
+
+    The C entry points receive only pointers and these sizes, and the kernels' tensor maps span
+    exactly those sizes: a k or v smaller than q implies would be read past its end, so every
+    shape is checked against q's here."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dim() != 4:
+            raise ValueError(f"{n} must be 4-D [B, heads, length, dim], got shape {tuple(t.shape)}")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    _shape(k, "k", (B, Hkv, Lk, d))
+    ldv = v.shape[-1]
+    _shape(v, "v", (B, Hkv, Lk, ldv))
+    return B, Hq, Lq, d, Hkv, Lk, ldv
+
+
+def _outputs(out, lse, shape_o, shape_l, dtype, device, want_lse=True):
+    """Caller-given or fresh O (``dtype``) and LSE (fp32) buffers, checked against their shapes."""
+    if out is None:
+        out = torch.empty(shape_o, dtype=dtype, device=device)
+    _need(out, "out", dtype)
+    _shape(out, "out", shape_o)
+    if lse is None and want_lse:
+        lse = torch.empty(shape_l, dtype=torch.float32, device=device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32)
+        _shape(lse, "lse", shape_l)
+    _same_device("outputs", out, lse)
+    if out.device != torch.device(device):
+        raise ValueError(f"out is on {out.device}, the inputs on {device}")
+    return out, lse
+
+
 def _elem_code(q: torch.Tensor) -> int:
     if q.dtype not in _DTYPE_CODE:
         raise ValueError(f"q must be bfloat16 or float16, got {q.dtype}")
@@ -114,18 +159,14 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
     code_t = _elem_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
-    B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    dv = v.shape[-1]
+    _same_device("attn_fwd", q, k, v)
+    B, Hq, Lq, d, Hkv, Lk, dv = _qkv_dims(q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
-    _need(out, "out", q.dtype)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_fwd_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
-                               scale, int(bool(causal)), code_t, _stream_handle(q.device))
+    out, lse = _outputs(out, lse, (B, Hq, Lq, dv), (B, Hq, Lq), q.dtype, q.device, want_lse)
+    with torch.cuda.device(q.device):
+        code = _lib.attn_fwd_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Lq, Lk, d, dv,
+                                   scale, int(bool(causal)), code_t, _stream_handle(q.device))
     _check(code, "attn_fwd")
     return out, lse
 
@@ -143,21 +184,17 @@ def attn_fwd_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_idx
         _need(t, n, q.dtype)
     _need(block_idx, "block_idx", torch.int32)
     _need(block_cnt, "block_cnt", torch.int32)
-    B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    dv = v.shape[-1]
+    _same_device("attn_fwd_sparse", q, k, v, block_idx, block_cnt)
+    B, Hq, Lq, d, Hkv, Lk, dv = _qkv_dims(q, k, v)
     nqb = (Lq + SPARSE_BLOCK - 1) // SPARSE_BLOCK
     if block_cnt.shape != (B, Hq, nqb) or block_idx.dim() != 4 or block_idx.shape[:3] != (B, Hq, nqb):
         raise ValueError(f"block lists must be [B, Hq, {nqb}, max_blocks] and [B, Hq, {nqb}]")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
-    _need(out, "out", q.dtype)
-    if lse is None:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_fwd_sparse_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                      B, Hq, Hkv, Lq, Lk, d, dv, scale, int(bool(causal)), block_idx.data_ptr(),
-                                      block_cnt.data_ptr(), block_idx.shape[3], code_t, _stream_handle(q.device))
+    out, lse = _outputs(out, lse, (B, Hq, Lq, dv), (B, Hq, Lq), q.dtype, q.device)
+    with torch.cuda.device(q.device):
+        code = _lib.attn_fwd_sparse_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                          B, Hq, Hkv, Lq, Lk, d, dv, scale, int(bool(causal)), block_idx.data_ptr(),
+                                          block_cnt.data_ptr(), block_idx.shape[3], code_t, _stream_handle(q.device))
     _check(code, "attn_fwd_sparse")
     return out, lse
 
@@ -178,23 +215,23 @@ def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bo
     code_t = _elem_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
-    B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    ldv = v.shape[-1]
+    _same_device("attn_decode", q, k, v, workspace)
+    B, Hq, Lq, d, Hkv, Lk, ldv = _qkv_dims(q, k, v)
     dv = ldv if dv is None else int(dv)
+    if not 1 <= dv <= ldv:
+        raise ValueError(f"dv = {dv} must be in [1, {ldv}] (the width of v)")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     need = attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=q.device)
-    _need(out, "out", q.dtype)
-    if lse is None:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_decode_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                  B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, int(bool(causal)), int(num_splits),
-                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(impl),
-                                  code_t, _stream_handle(q.device))
+    elif not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    out, lse = _outputs(out, lse, (B, Hq, Lq, dv), (B, Hq, Lq), q.dtype, q.device)
+    with torch.cuda.device(q.device):
+        code = _lib.attn_decode_typed(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, int(bool(causal)), int(num_splits),
+                                      workspace.data_ptr(), workspace.numel() * workspace.element_size(), int(impl),
+                                      code_t, _stream_handle(q.device))
     _check(code, "attn_decode")
     return out, lse
 
@@ -207,14 +244,17 @@ def attn_combine(o_part: torch.Tensor, lse_part: torch.Tensor, *, B: int, Hq: in
     _need(lse_part, "lse_part", torch.float32)
     if dtype not in _DTYPE_CODE:
         raise ValueError(f"dtype must be bfloat16 or float16, got {dtype}")
+    if o_part.dim() != 3:
+        raise ValueError(f"o_part must be 3-D [splits, rows, dv], got shape {tuple(o_part.shape)}")
     S, rows, dv = o_part.shape
-    if out is None:
-        out = torch.empty((B, Hq, Lq, dv), dtype=dtype, device=o_part.device)
-    _need(out, "out", dtype)
-    if lse is None:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=o_part.device)
-    code = _lib.attn_combine_typed(o_part.data_ptr(), lse_part.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                   B, Hq, Lq, dv, S, _DTYPE_CODE[dtype], _stream_handle(o_part.device))
+    if rows != B * Hq * Lq:
+        raise ValueError(f"o_part has {rows} rows, B*Hq*Lq = {B * Hq * Lq}")
+    _shape(lse_part, "lse_part", (S, rows))
+    _same_device("attn_combine", o_part, lse_part)
+    out, lse = _outputs(out, lse, (B, Hq, Lq, dv), (B, Hq, Lq), dtype, o_part.device)
+    with torch.cuda.device(o_part.device):
+        code = _lib.attn_combine_typed(o_part.data_ptr(), lse_part.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                       B, Hq, Lq, dv, S, _DTYPE_CODE[dtype], _stream_handle(o_part.device))
     _check(code, "attn_combine")
     return out, lse
 
@@ -246,12 +286,20 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: 
     in on one stream, computed on a second and copied out on a third, so the host-to-device
     copies, the kernels and the device-to-host copies of different pieces overlap. ``bufs`` may
     hold the reusable device buffers, pinned outputs, streams and events between calls."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda:
+            raise ValueError(f"{n} must be a host tensor (pinned for overlapped copies)")
+        if t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous {q.dtype}")
+    B, Hq, Lq, d, Hkv, Lk, dv = _qkv_dims(q, k, v)
+    if Hq % Hkv != 0:
+        raise ValueError(f"Hq = {Hq} is not a multiple of Hkv = {Hkv}")
     dev = torch.device(device)
     bufs = {} if bufs is None else bufs
-    B, Hq, Lq, d = q.shape
-    _, Hkv, Lk, _ = k.shape
-    dv = v.shape[-1]
     G = Hq // Hkv
+    if "o" in bufs and any(bufs[n].shape != t.shape or bufs[n].dtype != t.dtype
+                           for n, t in (("q", q), ("k", k), ("v", v))):
+        raise ValueError("bufs holds buffers of another shape or dtype; pass a fresh dict")
     if "o" not in bufs:
         for name, t in (("q", q), ("k", k), ("v", v)):
             bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)

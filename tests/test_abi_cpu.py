@@ -277,3 +277,43 @@ def test_binding_argtypes_match_header():
             assert len(fn.argtypes) == n, f"{name}: header {n} parameters, binding {len(fn.argtypes)}"
             checked += 1
     assert checked >= 10
+
+
+def test_binding_checks_shapes_against_q():
+    """The C calls receive only pointers and q's sizes, so the binding rejects a k, v or output
+    whose shape disagrees (their tensor maps would otherwise reach past the end of the tensor)."""
+    import torch
+    from exact_attention_139_b200 import attn
+    q = torch.empty(2, 8, 300, 128, dtype=torch.bfloat16)
+    k = torch.empty(2, 2, 500, 128, dtype=torch.bfloat16)
+    v = torch.empty(2, 2, 500, 128, dtype=torch.bfloat16)
+    assert attn._qkv_dims(q, k, v) == (2, 8, 300, 128, 2, 500, 128)
+    assert attn._qkv_dims(q, k, k) == (2, 8, 300, 128, 2, 500, 128)  # latent: v is k
+    for bad_k in (torch.empty(1, 2, 500, 128), torch.empty(2, 2, 500, 64), torch.empty(2, 2, 500)):
+        with pytest.raises(ValueError):
+            attn._qkv_dims(q, bad_k, v)
+    for bad_v in (torch.empty(2, 2, 499, 128), torch.empty(2, 1, 500, 128), torch.empty(1, 2, 500, 128)):
+        with pytest.raises(ValueError):
+            attn._qkv_dims(q, k, bad_v)
+    with pytest.raises(ValueError):
+        attn._shape(torch.empty(2, 8, 300), "lse", (2, 8, 301))
+    attn._same_device("x", q, None, k)
+    with pytest.raises(ValueError):
+        attn._same_device("x", q, torch.empty(1, device="meta"))
+
+
+def test_host_path_checks_inputs_before_device_work():
+    """attn_fwd_host validates shapes and reused buffers before it touches a device."""
+    import torch
+    from exact_attention_139_b200 import attn
+    q = torch.empty(1, 4, 256, 128, dtype=torch.bfloat16)
+    k = torch.empty(1, 2, 256, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd_host(q, k, torch.empty(1, 2, 128, 128, dtype=torch.bfloat16), causal=True)
+    with pytest.raises(ValueError):
+        attn.attn_fwd_host(q, k, k.float(), causal=True)
+    with pytest.raises(ValueError):
+        attn.attn_fwd_host(torch.empty(1, 3, 256, 128, dtype=torch.bfloat16), k, k, causal=True)
+    stale = {"o": None, "q": torch.empty(1, 4, 128, 128, dtype=torch.bfloat16), "k": k, "v": k}
+    with pytest.raises(ValueError, match="another shape"):
+        attn.attn_fwd_host(q, k, k, causal=True, bufs=stale)

@@ -99,3 +99,26 @@ def test_host_path_matches_device_path(B, Hq, Hkv, chunks, cuda_device):
         o_h, l_h = attn.attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True,
                                       device=cuda_device, bufs=bufs, chunks=chunks)
         assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+
+
+def test_binding_rejects_mismatched_tensors(cuda_device):
+    """Shapes that disagree with q are refused in the binding, before anything is launched."""
+    from exact_attention_139_b200 import attn
+    bf = dict(dtype=torch.bfloat16, device=cuda_device)
+    q = torch.zeros(1, 4, 256, 128, **bf)
+    k = torch.zeros(1, 2, 256, 128, **bf)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, k, torch.zeros(1, 2, 128, 128, **bf), causal=True)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, k, k, causal=True, out=torch.empty(1, 4, 128, 128, **bf))
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, k, k, causal=True, lse=torch.empty(4, 256, dtype=torch.float32, device=cuda_device))
+    with pytest.raises(ValueError):
+        attn.attn_decode(q[:, :, :1].contiguous(), k, k, causal=True, dv=256)
+    op = torch.zeros(2, 8, 128, dtype=torch.float32, device=cuda_device)
+    with pytest.raises(ValueError):
+        attn.attn_combine(op, torch.zeros(2, 8, dtype=torch.float32, device=cuda_device), B=1, Hq=4, Lq=1)
+    with pytest.raises(ValueError):
+        attn.attn_combine(op, torch.zeros(2, 7, dtype=torch.float32, device=cuda_device), B=1, Hq=8, Lq=1)
+    o, _ = attn.attn_fwd(q, k, k, causal=True)  # the same call with matching shapes runs
+    assert attn.attn_check_device() == attn.ATTN_OK and o.shape == q.shape
