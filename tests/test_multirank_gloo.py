@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_max_time_and_independent_batches():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
@@ -113,7 +113,7 @@ def test_two_ranks_head_shards_reassemble_the_layer():
     from oracle import oracle
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
