@@ -44,6 +44,8 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # roofline "traffic". Re-measure whenever one of these kernels changes.
 NCU_TRAFFIC_BYTES = {
     "llama8b_prefill_8k": 132.6e6,   # prefill2_kernel<128, bf16, dense>
+    "batched_prefill_2k": 787.4e6,   # same kernel
+    "batched_prefill_256": 51.7e6,   # same kernel (O still in L2 when it ends)
     "mla_decode_64k": 2427.1e6,      # decode_tn_kernel<9,2,48,3,latent,bf16>, balanced grid
     "gqa_decode_32k": 2154.3e6,      # decode_tn_kernel<2,1,48,3,dense V,bf16>, balanced grid
 }
@@ -373,7 +375,8 @@ def run_ours(args):
             "ms_per_step": round(shms, 4),
             "roofline": {"bound": "max(tensor, hbm)", "achieved_ms": round(shms, 4), "bound_ms": round(t_bound * 1e3, 4),
                          "frac": round(t_bound * 1e3 / shms, 4), "algorithmic_flops_per_launch": wsh.flops(),
-                         "algorithmic_bytes_per_launch": sh_bytes}}
+                         "algorithmic_bytes_per_launch": sh_bytes,
+                         "traffic": NCU_TRAFFIC_BYTES.get(wsh.name) if world == 1 or args.shard == "batch" else None}}
         launches += args.steps
         if not args.no_f16:
             # fp16 inputs: same kernels with the fp16 operand format; fp16 and bf16 share one
