@@ -159,6 +159,9 @@ static int listed(const problem *p, int64_t b, int64_t h, int64_t i, int64_t j) 
 static int visible(const problem *p, int64_t b, int64_t h, int64_t i, int64_t j) {
     if (j < p->kv_begin || j >= p->kv_end) return 0;
     if (!listed(p, b, h, i, j)) return 0;
+#if ORACLE_MUTANT == 14
+    if (p->blk_cnt) return 1; /* planted: a listed block bypasses the causal rule */
+#endif
     if (!p->causal) return 1;
 #if ORACLE_MUTANT == 4
     return j <= i; /* planted: top-left alignment */
@@ -405,6 +408,15 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
         for (int64_t j = 0; j < Lk; ++j) St[j * Lq + i] /= l;
         lse[i] = m + log(l);
     }
+#if ORACLE_MUTANT == 12
+    /* planted: each key's probabilities renormalised over the queries (the wrong axis of P^T) */
+    for (int64_t j = 0; j < Lk; ++j) {
+        double t = 0.0;
+        for (int64_t i = 0; i < Lq; ++i) t += St[j * Lq + i];
+        if (t > 0.0)
+            for (int64_t i = 0; i < Lq; ++i) St[j * Lq + i] /= t;
+    }
+#endif
     /* Ot[c][i] = sum_j V[j][c] * Pt[j][i] */
     for (int64_t c = 0; c < dv; ++c)
         for (int64_t i = 0; i < Lq; ++i) {
@@ -415,7 +427,12 @@ int oracle_attn_transposed_head(const uint16_t *q, const uint16_t *k, const uint
         }
     /* O = Ot^T */
     for (int64_t i = 0; i < Lq; ++i)
-        for (int64_t c = 0; c < dv; ++c) o[i * dv + c] = Ot[c * Lq + i];
+        for (int64_t c = 0; c < dv; ++c)
+#if ORACLE_MUTANT == 13
+            o[i * dv + c] = Ot[i * dv + c]; /* planted: the final transpose left out */
+#else
+            o[i * dv + c] = Ot[c * Lq + i];
+#endif
     free(St);
     free(Ot);
     return 0;
@@ -448,7 +465,11 @@ int oracle_combine(const double *o_parts, const double *lse_parts, int64_t n_spl
         for (int64_t s = 0; s < n_splits; ++s) {
             double ls = lse_parts[s * n_rows + r];
             if (ls == -INFINITY) continue;
+#if ORACLE_MUTANT == 11
+            double w = exp(ls - m); /* planted: weights not divided by the sum over splits */
+#else
             double w = exp(ls - L);
+#endif
             for (int64_t c = 0; c < dv; ++c) o[r * dv + c] += w * o_parts[(s * n_rows + r) * dv + c];
         }
     }
