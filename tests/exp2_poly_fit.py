@@ -4,7 +4,7 @@ FMA pipe instead of the MUFU unit.
 2^x = 2^n * 2^f with n = round(x) and f = x - n in [-0.5, 0.5]; 2^f is approximated by the degree-3
 polynomial that minimises the maximum relative error on [-0.5, 0.5], found with the Remez exchange
 algorithm (E. Remez, 1934). Running this file prints the coefficients rounded to fp32 and the error
-of the fp32 Horner evaluation; csrc/sm100.cuh holds the same four numbers (a CPU test checks that
+of the fp32 Horner evaluation; exact_attention_139_b200/csrc/sm100.cuh holds the same four numbers (a CPU test checks that
 they match this fit and the bound).
 """
 from __future__ import annotations

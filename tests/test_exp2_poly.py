@@ -6,7 +6,7 @@ import re
 import numpy as np
 import pytest
 
-from exact_attention_139_b200 import exp2_poly_fit
+from tests import exp2_poly_fit
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
