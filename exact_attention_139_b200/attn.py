@@ -12,7 +12,7 @@ taken from q (the C ``*_typed`` entry points receive it):
     attn_combine(o_part, lse_part, out=None, lse=None, dtype=bf16)         -> (o, lse)
     attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits)         -> int
     attn_status_string(code), attn_check_device(), attn_selftest_wait_timeout(limit_us)
-plus attn_fwd_host(...): host tensors in, host tensors out (pinned copies around attn_fwd).
+plus attn_fwd_host(...): host tensors in, host tensors out (the C attn_fwd_host pipeline).
 """
 from __future__ import annotations
 
@@ -48,8 +48,12 @@ _lib.attn_combine.restype = _i
 _lib.attn_combine.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 5 + [_vp]
 _lib.attn_combine_typed.restype = _i
 _lib.attn_combine_typed.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp]
+_lib.attn_fwd_host.restype = _i
+_lib.attn_fwd_host.argtypes = [_vp, _vp, _vp, _vp, _vp] + [_i] * 7 + [_f, _i, _i, _vp, _sz, _i, _vp]
+_lib.attn_fwd_host_scratch_size.restype = _sz
+_lib.attn_fwd_host_scratch_size.argtypes = [_i] * 7
 _lib.attn_decode_default_splits.restype = _i
-_lib.attn_decode_default_splits.argtypes = [_i] * 7
+_lib.attn_decode_default_splits.argtypes = [_i] * 8
 _lib.attn_check_device.restype = _i
 _lib.attn_check_device.argtypes = [_vp]
 _lib.attn_selftest_wait_timeout.restype = _i
@@ -203,8 +207,8 @@ def attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits=0) -> int:
     return int(_lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, num_splits))
 
 
-def attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv) -> int:
-    return int(_lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv))
+def attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv, latent: bool) -> int:
+    return int(_lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv, int(latent)))
 
 
 def attn_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
@@ -270,22 +274,12 @@ def attn_selftest_wait_timeout(limit_us: int, device=None):
     _check(_lib.attn_selftest_wait_timeout(int(limit_us), _stream_handle(dev)), "attn_selftest_wait_timeout")
 
 
-def _host_chunks(B: int, Hkv: int, want: int):
-    """(b, kv0, kv1) pieces of the [B, Hkv] unit grid, each inside one batch so that its q, k, v,
-    o and lse rows are contiguous in memory; about `want` pieces in total."""
-    per_b = max(1, -(-want // B))
-    step = max(1, -(-Hkv // per_b))
-    return [(b, k0, min(Hkv, k0 + step)) for b in range(B) for k0 in range(0, Hkv, step)]
-
-
 def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, scale: float | None = None,
-                  device="cuda:0", bufs: dict | None = None, chunks: int = 4):
-    """Host (CPU, pinned) tensors in, host tensors out: copy in, attn_fwd, copy out, pipelined.
-
-    The (batch, kv head) grid is cut into about ``chunks`` contiguous pieces; piece i is copied
-    in on one stream, computed on a second and copied out on a third, so the host-to-device
-    copies, the kernels and the device-to-host copies of different pieces overlap. ``bufs`` may
-    hold the reusable device buffers, pinned outputs, streams and events between calls."""
+                  device="cuda:0", bufs: dict | None = None, pieces: int = 0):
+    """Host (CPU, pinned) tensors in, host tensors out, through the C entry point attn_fwd_host
+    (copy-in, compute and copy-out pipelined over pieces of the (batch, kv head) grid inside the
+    library). ``bufs`` may hold the device scratch and the pinned outputs between calls. Waits for
+    the call to finish (the returned host tensors are then valid)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if t.is_cuda:
             raise ValueError(f"{n} must be a host tensor (pinned for overlapped copies)")
@@ -296,46 +290,23 @@ def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: 
         raise ValueError(f"Hq = {Hq} is not a multiple of Hkv = {Hkv}")
     dev = torch.device(device)
     bufs = {} if bufs is None else bufs
-    G = Hq // Hkv
-    if "o" in bufs and any(bufs[n].shape != t.shape or bufs[n].dtype != t.dtype
-                           for n, t in (("q", q), ("k", k), ("v", v))):
+    key = (tuple(q.shape), tuple(k.shape), tuple(v.shape), q.dtype)
+    if "key" in bufs and bufs["key"] != key:
         raise ValueError("bufs holds buffers of another shape or dtype; pass a fresh dict")
-    if "o" not in bufs:
-        for name, t in (("q", q), ("k", k), ("v", v)):
-            bufs[name] = torch.empty(t.shape, dtype=t.dtype, device=dev)
-        bufs["o"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, device=dev)
-        bufs["lse"] = torch.empty((B, Hq, Lq), dtype=torch.float32, device=dev)
+    if "key" not in bufs:
+        nbytes = int(_lib.attn_fwd_host_scratch_size(B, Hq, Hkv, Lq, Lk, d, dv))
+        if nbytes == 0:
+            raise ValueError("invalid sizes")
+        bufs["key"] = key
+        bufs["scratch"] = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         bufs["o_host"] = torch.empty((B, Hq, Lq, dv), dtype=q.dtype, pin_memory=True)
         bufs["lse_host"] = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
-        bufs["streams"] = [torch.cuda.Stream(dev) for _ in range(3)]
-    s_in, s_run, s_out = bufs["streams"]
-    main = torch.cuda.current_stream(dev)
-    s_in.wait_stream(main)  # earlier work on the caller's stream (e.g. a previous call) comes first
-    dq, dk, dvv, do, dl = bufs["q"], bufs["k"], bufs["v"], bufs["o"], bufs["lse"]
-    pieces = _host_chunks(B, Hkv, chunks)
-    done_out = []
-    for b, k0, k1 in pieces:
-        h0, h1 = k0 * G, k1 * G
-        e_in = torch.cuda.Event()
-        with torch.cuda.stream(s_in):
-            dq[b, h0:h1].copy_(q[b, h0:h1], non_blocking=True)
-            dk[b, k0:k1].copy_(k[b, k0:k1], non_blocking=True)
-            dvv[b, k0:k1].copy_(v[b, k0:k1], non_blocking=True)
-            e_in.record(s_in)
-        e_run = torch.cuda.Event()
-        with torch.cuda.stream(s_run):
-            s_run.wait_event(e_in)
-            attn_fwd(dq[b:b + 1, h0:h1], dk[b:b + 1, k0:k1], dvv[b:b + 1, k0:k1], causal=causal, scale=scale,
-                     out=do[b:b + 1, h0:h1], lse=dl[b:b + 1, h0:h1])
-            e_run.record(s_run)
-        e_out = torch.cuda.Event()
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(e_run)
-            bufs["o_host"][b, h0:h1].copy_(do[b, h0:h1], non_blocking=True)
-            bufs["lse_host"][b, h0:h1].copy_(dl[b, h0:h1], non_blocking=True)
-            e_out.record(s_out)
-        done_out.append(e_out)
-    for e in done_out:
-        main.wait_event(e)
-    main.synchronize()
+    sc = scale if scale is not None else 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        _check(_lib.attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), bufs["o_host"].data_ptr(),
+                                  bufs["lse_host"].data_ptr(), B, Hq, Hkv, Lq, Lk, d, dv, sc, int(bool(causal)),
+                                  _elem_code(q), bufs["scratch"].data_ptr(), bufs["scratch"].numel(),
+                                  int(pieces), stream.cuda_stream), "attn_fwd_host")
+    stream.synchronize()
     return bufs["o_host"], bufs["lse_host"]

@@ -19,7 +19,7 @@ ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 def _sources():
     return (glob.glob(os.path.join(PKG, "csrc", "*.cu")) + glob.glob(os.path.join(PKG, "csrc", "*.cuh"))
-            + [os.path.join(ROOT, "include", "attn.h")])
+            + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def _nvcc() -> str:

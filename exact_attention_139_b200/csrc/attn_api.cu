@@ -1,4 +1,5 @@
-// attn_api.cu -- the C ABI of libattn_b200.so (declared in include/attn.h).
+// attn_api.cu -- the C ABI of libattn_b200.so (declared in include/attn.h and, for the
+// diagnostics, include/attn_diag.h).
 //
 // Host side only: argument checks, TMA tensor-map encoding (driver entry point looked up once),
 // split selection and kernel launches. The kernels live in the .cuh files included below so the
@@ -13,15 +14,17 @@
 #include <cuda_runtime.h>
 
 #include "../../include/attn.h"
+#include "../../include/attn_diag.h"
 #include "combine.cuh"
 #include "decode.cuh"
 #include "prefill2.cuh"
+#include "prefill_pair.cuh"
 
 namespace {
 
 using attn::DecodeParams;
 
-constexpr int kAbiVersion = 10200;  // 1.2.0: block-sparse forward (attn_fwd_sparse_typed)
+constexpr int kAbiVersion = 10300;  // 1.3.0: attn_decode_default_splits takes the KV layout
 
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -74,6 +77,24 @@ int current_sm_count() {
 template <typename K>
 bool allow_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// How many clusters of a kernel can be resident at once on the current device (queried once per
+// device and kernel; `fallback` when the query fails).
+template <typename K>
+int resident_clusters(K kernel, cudaLaunchConfig_t cfg, int fallback) {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return std::max(1, fallback);
+  if (cache[dev] > 0) return cache[dev];
+  cfg.gridDim = dim3(2u * (unsigned)std::max(1, fallback));
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return std::max(1, fallback);
+  }
+  cache[dev] = n;
+  return n;
 }
 
 attn_status launch_status() {
@@ -431,6 +452,35 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   p.max_blk = sb.max_blk;
   p.n_qblocks = n_qtiles;
   p.n_kblocks = (Lk + 127) / 128;
+#ifndef ATTN_PREFILL_PAIR
+#define ATTN_PREFILL_PAIR 0
+#endif
+  // d = 128, dense key ranges, even GQA groups: the kernel whose products span a pair of SMs
+  if (ATTN_PREFILL_PAIR && !SPARSE && d == 128 && (Hq / Hkv) % 2 == 0) {
+    CUtensorMap tkh;  // K in boxes of 64 keys: each CTA of a pair loads half of a key tile
+    if (!encode16<E>(&tkh, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 64)) return ATTN_ERR_CUDA;
+    const long long pair_units = (long long)p.n_pairs * B * (Hq / 2);
+    if (pair_units > 0x7fff0000LL) return ATTN_ERR_UNSUPPORTED;
+    p.n_units = (int)pair_units;
+    auto kern = attn::prefill_pair_kernel<E>;
+    if (!allow_smem(kern, attn::PairCfg::SMEM_BYTES)) return ATTN_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(attn::PairCfg::THREADS);
+    cfg.dynamicSmemBytes = attn::PairCfg::SMEM_BYTES;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent grid: as many pairs as can be resident at once (SM pairs must share a GPC)
+    const int pairs = (int)std::min<long long>(pair_units, resident_clusters(kern, cfg, current_sm_count() / 2));
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    if (cudaLaunchKernelEx(&cfg, kern, tq, tkh, tv, p) != cudaSuccess) return ATTN_ERR_CUDA;
+    return launch_status();
+  }
   // persistent grid: one CTA per SM (fewer when there are fewer work units)
   const int grid = (int)std::min<long long>(units, current_sm_count());
   if (d == 128) {
@@ -445,23 +495,30 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   return launch_status();
 }
 
-template <typename E>
-attn_status decode_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                        int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
-                        void* workspace, size_t ws_bytes, int impl, void* stream) {
+// Every argument check of a decode call that does not involve the workspace; on success *impl
+// holds the resolved kernel choice (ATTN_DECODE_AUTO replaced).
+attn_status check_decode(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
+                         int Hkv, int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                         int* impl) {
   attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
   if (st != ATTN_OK) return st;
   if (ldv < dv) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
-  if (impl < ATTN_DECODE_AUTO || impl > ATTN_DECODE_TCGEN05_N) return ATTN_ERR_INVALID_ARG;
+  if (*impl < ATTN_DECODE_AUTO || *impl > ATTN_DECODE_TCGEN05_N) return ATTN_ERR_INVALID_ARG;
   if (d % 8 != 0 || dv % 8 != 0 || ldv % 8 != 0) return ATTN_ERR_MISALIGNED;
-  const bool tc_ok = tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
-  const bool tn_ok = tn_supported(k, v, Hq, Hkv, Lq, d, dv, ldv);
-  const bool cc_ok = cc_supported(Hq, Hkv, Lq, d, dv, ldv);
-  if (impl == ATTN_DECODE_AUTO) impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
-  if (impl == ATTN_DECODE_TCGEN05_T && !tc_ok) return ATTN_ERR_UNSUPPORTED;
-  if (impl == ATTN_DECODE_TCGEN05_N && !tn_ok) return ATTN_ERR_UNSUPPORTED;
-  if (impl == ATTN_DECODE_CUDA_CORE && !cc_ok) return ATTN_ERR_UNSUPPORTED;
+  if (*impl == ATTN_DECODE_AUTO) *impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
+  if (*impl == ATTN_DECODE_TCGEN05_T && !tc_supported(k, v, Hq, Hkv, Lq, d, dv, ldv)) return ATTN_ERR_UNSUPPORTED;
+  if (*impl == ATTN_DECODE_TCGEN05_N && !tn_supported(k, v, Hq, Hkv, Lq, d, dv, ldv)) return ATTN_ERR_UNSUPPORTED;
+  if (*impl == ATTN_DECODE_CUDA_CORE && !cc_supported(Hq, Hkv, Lq, d, dv, ldv)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+template <typename E>
+attn_status decode_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Lq, int Lk, int d, int dv, int ldv, float scale, int causal, int num_splits,
+                        void* workspace, size_t ws_bytes, int impl, void* stream) {
+  attn_status st = check_decode(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits, &impl);
+  if (st != ATTN_OK) return st;
   const bool dense_v = !(v == k && ldv == d);
   const DecodePlan plan = plan_decode(impl, dense_v, B, Hq, Hkv, Lq, Lk, d, dv, num_splits);
   const int splits = plan.splits;
@@ -575,13 +632,14 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv
   return workspace_bytes((long long)B * Hq * Lq, dv, most);
 }
 
-int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return 0;
-  // the queries-on-M kernel serves R <= 32 rows per kv head; dv == d == 128 is taken to be a
-  // dense V (the GQA decode shape)
-  const int R = (Hq / Hkv) * Lq;
-  const int impl = R <= 32 ? ATTN_DECODE_TCGEN05_N : ATTN_DECODE_CUDA_CORE;
-  return plan_decode(impl, dv == d && d == 128, B, Hq, Hkv, Lq, Lk, d, dv, 0).splits;
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int latent) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || d < 1 || dv < 1 || Hq % Hkv != 0) return 0;
+  // the kernel attn_decode picks for this layout (pointers only matter as "v == k or not")
+  const void* k = reinterpret_cast<const void*>(uintptr_t(0x100));
+  const void* v = latent ? k : reinterpret_cast<const void*>(uintptr_t(0x200));
+  const int ldv = latent ? d : dv;
+  const int impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
+  return plan_decode(impl, !latent, B, Hq, Hkv, Lq, Lk, d, dv, 0).splits;
 }
 
 attn_status attn_decode_typed(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -620,21 +678,57 @@ namespace {
 static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Driver entry points used to tell contexts apart (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Set-up, done once per device: the device address of the scratch array, looked up with that
+// device current. The address belongs to the device's (primary) context; the lookup is tagged
+// with the context's unique id and repeated if the context has changed since (a cudaDeviceReset
+// destroys the context and its copy of the array, and the next context may place it elsewhere).
+struct ScratchAddr {
+  void* ptr;
+  unsigned long long ctx_id;
+};
+std::mutex g_scratch_mu;
+ScratchAddr g_scratch[kMaxDevices] = {};
+
 attn_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  // no current context yet (first runtime call on this thread): the lookup below creates it
+  unsigned long long ctx_id = 0;
+  const bool have_ctx = current_context_id(&ctx_id);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (!have_ctx || g_scratch[dev].ptr == nullptr || g_scratch[dev].ctx_id != ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    if (!current_context_id(&ctx_id)) return ATTN_ERR_CUDA;
+    g_scratch[dev] = ScratchAddr{p, ctx_id};
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return ATTN_OK;
 }
 
@@ -645,10 +739,10 @@ extern "C" {
 attn_status attn_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                                 int Hkv, int Lq, int Lk, int d, int dv, int ldv, float scale, int causal,
                                 int num_splits, void* stream) {
-  attn_status st = check_common(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  // the same checks, in the same order, as attn_decode's; only then the scratch size
+  int impl = ATTN_DECODE_AUTO;
+  attn_status st = check_decode(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, dv, ldv, scale, causal, num_splits, &impl);
   if (st != ATTN_OK) return st;
-  if (num_splits < 0 || num_splits > 256) return ATTN_ERR_INVALID_ARG;
-  const int impl = auto_impl(k, v, Hq, Hkv, Lq, d, dv, ldv);
   const DecodePlan plan = plan_decode(impl, !(v == k && ldv == d), B, Hq, Hkv, Lq, Lk, d, dv, num_splits);
   const size_t need = workspace_bytes((long long)B * Hq * Lq, dv, plan.splits);
   if (need > (size_t)ATTN_DECODE_NOALLOC_SCRATCH_BYTES) return ATTN_ERR_WORKSPACE;
@@ -692,6 +786,160 @@ attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
   const int threads = 256, pairs = (n + 1) / 2;
   selftest_exp2_kernel<<<(pairs + threads - 1) / threads, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
   return launch_status();
+}
+
+}  // extern "C"
+
+namespace {
+
+// ---------------------------------------------------------------------------------------------
+// Host-buffer forward: copy-in, compute and copy-out pipelined over pieces of the unit grid.
+// ---------------------------------------------------------------------------------------------
+constexpr int kHostMaxPieces = 64;
+
+// Per-device streams and events of the host pipeline, created on first use and kept for the
+// life of the process (streams and events hold no device memory). One mutex per device
+// serialises the host-side enqueue of concurrent calls, which share the events.
+struct HostPipe {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t e_entry = nullptr, e_done = nullptr;
+  cudaEvent_t e_in[kHostMaxPieces] = {}, e_run[kHostMaxPieces] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+bool host_pipe_init(HostPipe& hp) {
+  if (hp.ready) return true;
+  const unsigned ef = cudaEventDisableTiming;
+  if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&hp.e_entry, ef) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&hp.e_done, ef) != cudaSuccess) return false;
+  for (int i = 0; i < kHostMaxPieces; ++i)
+    if (cudaEventCreateWithFlags(&hp.e_in[i], ef) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.e_run[i], ef) != cudaSuccess)
+      return false;
+  hp.ready = true;
+  return true;
+}
+
+struct HostLayout {
+  size_t q, k, v, o, lse, total;  // byte offsets in the device scratch
+};
+
+HostLayout host_layout(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
+  HostLayout L{};
+  const size_t e = 2;  // 16-bit elements
+  L.q = 0;
+  L.k = align256(L.q + (size_t)B * Hq * Lq * d * e);
+  L.v = align256(L.k + (size_t)B * Hkv * Lk * d * e);
+  L.o = align256(L.v + (size_t)B * Hkv * Lk * dv * e);
+  L.lse = align256(L.o + (size_t)B * Hq * Lq * dv * e);
+  L.total = align256(L.lse + (size_t)B * Hq * Lq * 4);
+  return L;
+}
+
+// Piece boundaries over U units (unit = one (batch, kv head) with its G query heads). pieces > 0:
+// that many near-equal pieces (at most U). pieces == 0: three quarters in three equal pieces and
+// the last quarter in two halves, so the last kernel and its output copy (the drain after the
+// last input copy) are short while the first pieces stay large enough to keep the copies busy.
+int host_pieces(long long U, int pieces, long long* bounds) {
+  int n = 0;
+  bounds[0] = 0;
+  if (pieces > 0) {
+    n = (int)std::min<long long>(pieces, U);
+    for (int i = 1; i <= n; ++i) bounds[i] = U * i / n;
+    return n;
+  }
+  const long long qtr = (U + 3) / 4;
+  long long at = 0;
+  for (int i = 0; i < 3 && at < U; ++i) {
+    at = std::min(U, at + qtr);
+    bounds[++n] = at;
+  }
+  const long long rest = U - at;
+  if (rest > 1) bounds[++n] = at + (rest + 1) / 2;
+  if (rest > 0) bounds[++n] = U;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_fwd_host_scratch_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || d < 1 || dv < 1 || Hq % Hkv != 0) return 0;
+  return host_layout(B, Hq, Hkv, Lq, Lk, d, dv).total;
+}
+
+attn_status attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host, float* lse_host,
+                          int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, float scale, int causal, int dtype,
+                          void* scratch, size_t scratch_bytes, int pieces, void* stream) {
+  if (!valid_dtype(dtype)) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_common(q_host, k_host, v_host, o_host, lse_host, B, Hq, Hkv, Lq, Lk, d, dv, scale, causal);
+  if (st != ATTN_OK) return st;
+  if (d != dv || (d != 64 && d != 128)) return ATTN_ERR_UNSUPPORTED;
+  if (pieces < 0 || pieces > kHostMaxPieces) return ATTN_ERR_INVALID_ARG;
+  const HostLayout L = host_layout(B, Hq, Hkv, Lq, Lk, d, dv);
+  if (!scratch || scratch_bytes < L.total || !aligned(scratch, 256)) return ATTN_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  HostPipe& hp = g_host_pipe[dev];
+  std::lock_guard<std::mutex> lock(hp.mu);
+  if (!host_pipe_init(hp)) return ATTN_ERR_CUDA;
+
+  const int G = Hq / Hkv;
+  const long long U = (long long)B * Hkv;
+  long long bounds[kHostMaxPieces + 1];
+  const int n = host_pieces(U, pieces, bounds);
+  // bytes per unit of each tensor; a range of units is a contiguous range of every tensor
+  const size_t uq = (size_t)G * Lq * d * 2, uk = (size_t)Lk * d * 2, uv = (size_t)Lk * dv * 2;
+  const size_t uo = (size_t)G * Lq * dv * 2, ul = (size_t)G * Lq * 4;
+  uint8_t* base = reinterpret_cast<uint8_t*>(scratch);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  auto H2D = cudaMemcpyHostToDevice;
+  auto D2H = cudaMemcpyDeviceToHost;
+
+  // the copies start after earlier work on the caller's stream (e.g. a previous call's kernels,
+  // which read the same scratch)
+  if (cudaEventRecord(hp.e_entry, cs) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamWaitEvent(hp.s_in, hp.e_entry, 0) != cudaSuccess) return ATTN_ERR_CUDA;
+  for (int i = 0; i < n; ++i) {
+    const long long u0 = bounds[i], nu = bounds[i + 1] - bounds[i];
+    const uint8_t* qh = reinterpret_cast<const uint8_t*>(q_host);
+    const uint8_t* kh = reinterpret_cast<const uint8_t*>(k_host);
+    const uint8_t* vh = reinterpret_cast<const uint8_t*>(v_host);
+    if (cudaMemcpyAsync(base + L.q + u0 * uq, qh + u0 * uq, nu * uq, H2D, hp.s_in) != cudaSuccess ||
+        cudaMemcpyAsync(base + L.k + u0 * uk, kh + u0 * uk, nu * uk, H2D, hp.s_in) != cudaSuccess ||
+        cudaMemcpyAsync(base + L.v + u0 * uv, vh + u0 * uv, nu * uv, H2D, hp.s_in) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaEventRecord(hp.e_in[i], hp.s_in) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaStreamWaitEvent(cs, hp.e_in[i], 0) != cudaSuccess) return ATTN_ERR_CUDA;
+    // the piece is an attention problem of its own: nu "batches" of one kv head and G query heads
+    st = with_elem(dtype, [&](auto e) {
+      return fwd_impl<decltype(e), false>(base + L.q + u0 * uq, base + L.k + u0 * uk, base + L.v + u0 * uv,
+                                          base + L.o + u0 * uo, reinterpret_cast<float*>(base + L.lse + u0 * ul),
+                                          (int)nu, G, 1, Lq, Lk, d, scale, causal, SparseBlocks{nullptr, nullptr, 0},
+                                          stream);
+    });
+    if (st != ATTN_OK) return st;
+    if (cudaEventRecord(hp.e_run[i], cs) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaStreamWaitEvent(hp.s_out, hp.e_run[i], 0) != cudaSuccess) return ATTN_ERR_CUDA;
+    uint8_t* oh = reinterpret_cast<uint8_t*>(o_host);
+    if (cudaMemcpyAsync(oh + u0 * uo, base + L.o + u0 * uo, nu * uo, D2H, hp.s_out) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (lse_host) {
+      uint8_t* lh = reinterpret_cast<uint8_t*>(lse_host);
+      if (cudaMemcpyAsync(lh + u0 * ul, base + L.lse + u0 * ul, nu * ul, D2H, hp.s_out) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    }
+  }
+  // the caller's stream is ordered after the last output copy
+  if (cudaEventRecord(hp.e_done, hp.s_out) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamWaitEvent(cs, hp.e_done, 0) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 attn_status attn_check_device(void* stream) {

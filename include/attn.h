@@ -13,10 +13,10 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Pointers named q, k, v, o, lse, o_part, lse_part, workspace are DEVICE pointers owned by
- *    the caller. The library allocates no device memory, never synchronises, and returns as
- *    soon as the work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
- *    default stream).
+ *  - Pointers named q, k, v, o, lse, o_part, lse_part, workspace, scratch are DEVICE pointers
+ *    owned by the caller (names ending in _host are host pointers). The library allocates no
+ *    device memory, never synchronises, and returns as soon as the work is enqueued on `stream`
+ *    (a cudaStream_t passed as void*; NULL = legacy default stream).
  *  - Layouts are row-major and contiguous:
  *        q   [B, Hq,  Lq, d]   bf16 (or fp16, see the *_typed entry points)
  *        k   [B, Hkv, Lk, d]   same element type as q
@@ -37,8 +37,10 @@
  *    attn_check_device() reads (and clears); the kernel then stops early without hanging.
  *    Device-side index lists (attn_fwd_sparse_typed) that break their contract are recorded in
  *    a second device word (the kernel still finishes) and reported as ATTN_ERR_INVALID_ARG.
- *  - Thread safety: entry points keep no host state between calls except a once-per-process
- *    lookup of the driver's tensor-map encoder; concurrent calls on different streams are safe.
+ *  - Thread safety: entry points keep no host state between calls except once-per-process
+ *    lookups (the driver's tensor-map encoder, the resident-cluster count of a kernel) and the
+ *    per-device state named at attn_fwd_host and attn_decode_noalloc; concurrent calls on
+ *    different streams are safe.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -95,6 +97,41 @@ attn_status attn_fwd_typed(const void *q, const void *k, const void *v, void *o,
                            int causal, int dtype, void *stream);
 
 /*
+ * attn_fwd_host -- attn_fwd_typed on HOST buffers: the inputs are copied to the device, the
+ * attention is computed and O and LSE are copied back, all enqueued asynchronously.
+ *
+ * The (batch, kv head) grid is cut into pieces of consecutive units (a unit is one kv head of
+ * one batch with its Hq/Hkv query heads; a run of units is a contiguous range of q, k, v, o and
+ * lse, so each piece is one copy per tensor and one attn_fwd call of its own). Piece i is copied
+ * in on a library-owned stream, computed on `stream` and copied out on a second library-owned
+ * stream, so the host-to-device copies, the kernels and the device-to-host copies of different
+ * pieces overlap. The copies go over the host link, which is the bound of this call.
+ *   q_host, k_host, v_host   HOST inputs in the layouts of attn_fwd; page-locked (pinned) memory
+ *                           is needed for the copies to overlap (pageable memory works but the
+ *                           copies then serialise).
+ *   o_host, lse_host         HOST outputs (lse_host may be NULL); valid once `stream` has
+ *                           completed the call (e.g. after cudaStreamSynchronize(stream)).
+ *   scratch                  DEVICE buffer owned by the caller, 256-byte aligned, at least
+ *                           attn_fwd_host_scratch_size(...) bytes: the device copies of q, k, v,
+ *                           o and lse. Its contents on entry do not matter.
+ *   pieces                   0: the library's split (three equal pieces over three quarters of
+ *                           the units, the last quarter in two halves, so that the drain after
+ *                           the last input copy is short); 1..64: that many near-equal pieces
+ *                           (fewer if there are fewer units).
+ * The call is ordered after earlier work on `stream`, and later work on `stream` is ordered
+ * after its last copy. The library creates its two copy streams and its events on the first call
+ * on each device and keeps them until the process exits (they hold no device memory); concurrent
+ * calls on one device enqueue one after the other. Other arguments, checks and supported shapes
+ * are those of attn_fwd_typed; a scratch that is NULL, too small or misaligned gives
+ * ATTN_ERR_WORKSPACE.
+ */
+size_t attn_fwd_host_scratch_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv);
+attn_status attn_fwd_host(const void *q_host, const void *k_host, const void *v_host, void *o_host,
+                          float *lse_host, int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv,
+                          float scale, int causal, int dtype, void *scratch, size_t scratch_bytes,
+                          int pieces, void *stream);
+
+/*
  * attn_fwd_sparse_typed -- block-sparse forward attention over caller-given index lists.
  *
  * The MInference article (7minutos.es, on sparse attention for long-context prefill) describes
@@ -126,6 +163,10 @@ attn_status attn_fwd_sparse_typed(const void *q, const void *k, const void *v, v
  * shape and split count (num_splits = 0: the count attn_decode chooses on this device).
  * Layout of the workspace: o_part fp32 [num_splits, B*Hq*Lq, dv] followed (256-byte
  * aligned) by lse_part fp32 [num_splits, B*Hq*Lq]. Returns 0 for invalid sizes.
+ * Hkv and Lk are arguments (a plain split count would need only B, Hq, Lq and dv) because with
+ * num_splits = 0 the library plans the splits itself from the number of (batch, kv head) units
+ * B*Hkv and the key length Lk: the balanced schedule cuts the B*Hkv*Lk keys into one run per SM
+ * slot, and the partial count of a kv head follows from where those runs fall.
  */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int dv,
                                   int num_splits);
@@ -200,7 +241,9 @@ attn_status attn_decode_typed(const void *q, const void *k, const void *v, void 
  *     smaller num_splits or use attn_decode with a caller workspace.
  *   - The first call on each device looks up the device address of the scratch array (a
  *     synchronous host call that may load the library's GPU code). Make that first call before
- *     any stream capture on that device.
+ *     any stream capture on that device. The address is kept per device together with the id
+ *     of the CUDA context it belongs to; after a cudaDeviceReset (a new context) the next call
+ *     looks it up again, so that call too must come before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents. The kernels write
  *     every scratch byte they later read, so nothing needs clearing between calls, but two
  *     calls that overlap on the GPU (different streams, no ordering between them) race on the
@@ -213,7 +256,11 @@ attn_status attn_decode_noalloc(const void *q, const void *k, const void *v, voi
                                 float scale, int causal, int num_splits, void *stream);
 
 /*
- * attn_combine -- log-sum-exp merge of split partials over disjoint key ranges:
+ * attn_combine -- log-sum-exp merge of split partials over disjoint key ranges. Flash attention
+ * updates its softmax statistics "iteratively and locally", block by block ("Activar Flash
+ * Attention con llama.cpp", section "Que es Flash Attention"); merging the (max, sum, output)
+ * of two key chunks is that same update applied once more, written here with the log-sum-exp
+ * of each chunk:
  *   LSE = ln sum_s exp(lse_s),  O = sum_s exp(lse_s - LSE) * O_s   (splits with lse_s = -inf
  *   carry no weight). o_part fp32 [num_splits, rows, dv], lse_part fp32 [num_splits, rows],
  *   rows = B*Hq*Lq in [B, Hq, Lq] order; o bf16 [rows, dv]; lse fp32 [rows] (may be NULL).
@@ -228,10 +275,10 @@ attn_status attn_combine_typed(const float *o_part, const float *lse_part, void 
                                void *stream);
 
 /* Number of partial results per (batch, kv head) that attn_decode uses with num_splits = 0 on the
- * current device (the most any kv head gets under the balanced schedule). The shape is taken
- * to have a dense V when dv == d == 128, latent KV otherwise; attn_decode_workspace_size with
- * num_splits = 0 covers every case. */
-int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv);
+ * current device (the most any kv head gets under the balanced schedule) for a call with these
+ * sizes. latent != 0: MLA latent KV (v == k, ldv == d, V the first dv columns of each K row);
+ * latent == 0: a separate dense V. Returns 0 for invalid sizes. */
+int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, int dv, int latent);
 
 /*
  * attn_check_device -- synchronises `stream`, then reads and clears the device-side error
@@ -241,25 +288,6 @@ int attn_decode_default_splits(int B, int Hq, int Hkv, int Lq, int Lk, int d, in
  * compute entry points never synchronise.
  */
 attn_status attn_check_device(void *stream);
-
-/*
- * attn_selftest_wait_timeout -- diagnostic: launches one CTA that waits on a shared-memory
- * barrier nothing ever arrives on, with a wall-clock limit of `limit_us` microseconds
- * (1..1000000). The wait runs out, the kernel records ATTN_ERR_TIMEOUT in the device error word
- * and returns; the CUDA context stays usable. Pair with attn_check_device() to observe the
- * status. Enqueued on `stream`; returns ATTN_ERR_INVALID_ARG for a limit outside the range.
- */
-attn_status attn_selftest_wait_timeout(unsigned int limit_us, void *stream);
-
-/*
- * attn_selftest_exp2 -- diagnostic: y[i] = 2^x[i] for n device floats, computed with the FMA-pipe
- * polynomial the prefill softmax uses for part of its exponentials (round-to-nearest range
- * reduction, degree-3 minimax polynomial; relative error below 1e-4 for x in [-125, 64]; for x
- * below -126, -inf included, the result is exactly 0; between -126 and -125 it is tiny but not
- * accurate).
- * x and y are device pointers; enqueued on `stream`.
- */
-attn_status attn_selftest_exp2(const float *x, float *y, int n, void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *attn_status_string(attn_status status);

@@ -14,6 +14,7 @@ from exact_attention_139_b200 import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "attn.h")
+HEADERS = [HEADER, os.path.join(ROOT, "include", "attn_diag.h")]
 
 OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA, TIMEOUT = range(7)
 A = 0x10000  # 256-byte aligned fake device address
@@ -23,7 +24,7 @@ D_ = 0x40000
 
 
 def header_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(attn_\w+)\s*\(", text)))
 
@@ -57,7 +58,7 @@ def test_header_declares_expected_entry_points():
 
 def test_library_exports_every_header_symbol(lib):
     for name in header_functions():
-        assert hasattr(lib, name), f"{name} declared in attn.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
 
 
 def test_status_strings(lib):
@@ -68,7 +69,7 @@ def test_status_strings(lib):
         seen.add(s)
     assert len(seen) == 7
     assert lib.attn_status_string(99).decode() == "unknown status"
-    assert lib.attn_abi_version() == 10200
+    assert lib.attn_abi_version() == 10300
 
 
 def fwd(lib, q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128, scale=0.1,
@@ -195,10 +196,11 @@ def test_typed_entry_points_reject_unknown_dtype(lib, bad):
 
 def test_default_workspace_covers_default_splits(lib):
     """num_splits = 0 sizes the workspace for whichever split count attn_decode will choose."""
-    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 7
-    for B, Hq, Hkv, Lq, Lk, d, dv in [(16, 32, 8, 1, 32768, 128, 128), (32, 16, 1, 2, 65536, 576, 512),
-                                      (2, 8, 2, 1, 777, 128, 128), (4, 16, 2, 2, 5000, 256, 256)]:
-        s = lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv)
+    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 8
+    for B, Hq, Hkv, Lq, Lk, d, dv, lat in [(16, 32, 8, 1, 32768, 128, 128, 0), (32, 16, 1, 2, 65536, 576, 512, 1),
+                                           (2, 8, 2, 1, 777, 128, 128, 0), (4, 16, 2, 2, 5000, 256, 256, 0),
+                                           (8, 16, 1, 1, 9000, 128, 128, 1), (3, 4, 1, 2, 3000, 576, 512, 0)]:
+        s = lib.attn_decode_default_splits(B, Hq, Hkv, Lq, Lk, d, dv, lat)
         assert 1 <= s <= 256
         assert lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, 0) >= \
             lib.attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk, dv, s)
@@ -239,16 +241,16 @@ def _balanced_pieces(units, Lk, slots):
 def test_decode_plan_balanced_schedule(lib):
     """Without a GPU the library assumes 148 SMs; the latent kernel runs one CTA per SM, the dense
     d = 128 kernel two."""
-    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 7
-    mla = lib.attn_decode_default_splits(32, 16, 1, 2, 65536, 576, 512)
+    lib.attn_decode_default_splits.argtypes = [ctypes.c_int] * 8
+    mla = lib.attn_decode_default_splits(32, 16, 1, 2, 65536, 576, 512, 1)
     assert mla == _balanced_pieces(32, 65536, 148)
-    gqa = lib.attn_decode_default_splits(16, 32, 8, 1, 32768, 128, 128)
+    gqa = lib.attn_decode_default_splits(16, 32, 8, 1, 32768, 128, 128, 0)
     assert gqa == _balanced_pieces(128, 32768, 296)
-    odd = lib.attn_decode_default_splits(3, 16, 1, 2, 4097, 576, 512)
+    odd = lib.attn_decode_default_splits(3, 16, 1, 2, 4097, 576, 512, 1)
     assert odd == _balanced_pieces(3, 4097, 148)
     # many short kv heads: a run would span more than two heads, so equal chunks are used
     assert _balanced_pieces(64 * 8, 100, 296) is None
-    s = lib.attn_decode_default_splits(64, 32, 8, 1, 100, 128, 128)
+    s = lib.attn_decode_default_splits(64, 32, 8, 1, 100, 128, 128, 0)
     assert 1 <= s <= 256
     for (B, Hq, Hkv, Lq, Lk, d, dv), pieces in [((32, 16, 1, 2, 65536, 576, 512), mla),
                                                  ((16, 32, 8, 1, 32768, 128, 128), gqa),
@@ -258,7 +260,7 @@ def test_decode_plan_balanced_schedule(lib):
 
 
 def _header_param_counts():
-    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"/\*.*?\*/", "", "".join(open(h).read() for h in HEADERS), flags=re.S)
     out = {}
     for name, params in re.findall(r"\b(attn_\w+)\s*\(([^)]*)\)\s*;", text):
         params = params.strip()
@@ -314,6 +316,34 @@ def test_host_path_checks_inputs_before_device_work():
         attn.attn_fwd_host(q, k, k.float(), causal=True)
     with pytest.raises(ValueError):
         attn.attn_fwd_host(torch.empty(1, 3, 256, 128, dtype=torch.bfloat16), k, k, causal=True)
-    stale = {"o": None, "q": torch.empty(1, 4, 128, 128, dtype=torch.bfloat16), "k": k, "v": k}
+    stale = {"key": ((1, 4, 128, 128), tuple(k.shape), tuple(k.shape), torch.bfloat16)}
     with pytest.raises(ValueError, match="another shape"):
         attn.attn_fwd_host(q, k, k, causal=True, bufs=stale)
+
+
+def test_host_entry_point_argument_checks(lib):
+    """attn_fwd_host rejects bad arguments before touching a device (fake addresses)."""
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd_host.argtypes = [vp] * 5 + [i] * 7 + [f, i, i, vp, sz, i, vp]
+    lib.attn_fwd_host_scratch_size.argtypes = [i] * 7
+    lib.attn_fwd_host_scratch_size.restype = sz
+    need = lib.attn_fwd_host_scratch_size(1, 32, 8, 8192, 8192, 128, 128)
+    # q, k, v, o in 16-bit elements plus fp32 LSE, each 256-byte aligned
+    assert need == 2 * (2 * 32 * 8192 * 128 + 2 * 8 * 8192 * 128) + 32 * 8192 * 4
+    assert lib.attn_fwd_host_scratch_size(1, 3, 2, 10, 10, 64, 64) == 0
+
+    def host(**kw):
+        a = dict(q=A, k=B_, v=C_, o=D_, lse=None, B=1, Hq=2, Hkv=1, Lq=128, Lk=128, d=128, dv=128, scale=0.1,
+                 causal=1, dtype=0, scratch=0x100000, scratch_bytes=1 << 30, pieces=0)
+        a.update(kw)
+        return lib.attn_fwd_host(*a.values(), None)
+
+    assert host(q=None) == INVALID
+    assert host(dtype=5) == INVALID
+    assert host(pieces=-1) == INVALID
+    assert host(pieces=65) == INVALID
+    assert host(scratch=None) == WORKSPACE
+    assert host(scratch_bytes=1000) == WORKSPACE
+    assert host(scratch=0x100010) == WORKSPACE
+    assert host(d=96, dv=96) == UNSUPPORTED
+    assert host(Hq=3, Hkv=2) == INVALID

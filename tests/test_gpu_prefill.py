@@ -86,19 +86,35 @@ def test_deterministic(cuda_device):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,chunks", [(1, 32, 8, 4), (2, 4, 2, 4), (3, 2, 1, 1)])
-def test_host_path_matches_device_path(B, Hq, Hkv, chunks, cuda_device):
-    """attn_fwd_host (pinned host buffers, pieces pipelined over copy and compute streams) gives
-    the device call's O and LSE bit for bit."""
+@pytest.mark.parametrize("B,Hq,Hkv,pieces", [(1, 32, 8, 0), (1, 32, 8, 4), (2, 4, 2, 0), (2, 4, 2, 3),
+                                             (3, 2, 1, 1), (3, 2, 1, 64), (5, 6, 3, 0)])
+def test_host_path_matches_device_path(B, Hq, Hkv, pieces, cuda_device):
+    """attn_fwd_host (the C entry point: pinned host buffers, pieces pipelined over copy and
+    compute streams) gives the device call's O and LSE bit for bit."""
     from exact_attention_139_b200 import attn
     w = Workload("host", B, Hq, Hkv, 300, 300, 128, 128, True, seed=6000 + B)
     q, k, v = make_inputs(w)
     o_d, l_d = attn.attn_fwd(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), causal=True)
     bufs = {}
-    for _ in range(2):  # the second call reuses the buffers, streams and pinned outputs
+    for _ in range(2):  # the second call reuses the scratch and the pinned outputs
         o_h, l_h = attn.attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True,
-                                      device=cuda_device, bufs=bufs, chunks=chunks)
+                                      device=cuda_device, bufs=bufs, pieces=pieces)
         assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+    assert attn.attn_check_device() == attn.ATTN_OK
+
+
+def test_host_path_full_size_against_oracle(cuda_device):
+    """The 8K prefill through the host entry point, sampled rows against the oracle."""
+    from exact_attention_139_b200 import attn
+    w = WORKLOADS["llama8b_prefill_8k"]
+    q, k, v = make_inputs(w)
+    o_h, l_h = attn.attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), causal=True,
+                                  device=cuda_device)
+    assert attn.attn_check_device() == attn.ATTN_OK
+    rows = sample_rows(w, 32).numpy()
+    o_ref, l_ref = oracle_rows(w, q, k, v, rows)
+    og, lg = take_rows(o_h, l_h, rows)
+    compare(og, lg, o_ref, l_ref, "host path 8K")
 
 
 def test_binding_rejects_mismatched_tensors(cuda_device):
