@@ -53,9 +53,17 @@ struct Prefill2Params {
 #endif
 // Key pairs e (0..15 within each group of 32 keys) whose exponentials are computed with the FMA
 // polynomial (bit e set) instead of ex2.approx on the MUFU unit. One pair in eight measured best
-// on B200 (8K causal prefill: none 1116, 1/8 1135, 1/4 1099, 3/8 1093, 1/2 1071 TFLOP/s).
+// on B200 (8K causal prefill: none 1116, 1/8 1135, 1/4 1099, 3/8 1093, 1/2 1071 TFLOP/s; at
+// d = 64, where the exponentials weigh twice as much per tensor product, 1/8 651, 1/4 632,
+// 3/8 609, 1/2 538).
 constexpr uint32_t kExp2EmulateMask = ATTN_EXP2_EMULATE_MASK;
 
+// Shared memory: Q_A and Q_B, then a ring of NS stages, stage j holding K_j and V_j under one
+// full and one empty barrier; a stage is released by one commit after the last P.V product of its
+// tile. (Measured alternative: separate K and V rings, K three deep and V two deep, each slot
+// released after its last reader, so that K is fetched further ahead: same results, 3 % slower
+// at 8K and 2K. Cycle counters in the MMA-issuing thread showed that its waits for K and V took
+// under 4 % of its time either way: the loads are not what paces the kernel.)
 template <int D>
 struct Prefill2Cfg {
   static constexpr int BM = 128, BN = 128;
