@@ -423,8 +423,9 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                      int Lk, int d, float scale, int causal, SparseBlocks sb, void* stream) {
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int n_qtiles = (Lq + 127) / 128;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!encode16<E>(&tq, q, (uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
+      !encode16<E>(&to, o, (uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq, 64, 128) ||
       !encode16<E>(&tk, k, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128) ||
       !encode16<E>(&tv, v, (uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv, 64, 128))
     return ATTN_ERR_CUDA;
@@ -438,7 +439,10 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   p.Lk = Lk;
   p.G = Hq / Hkv;
   p.n_pairs = (n_qtiles + 1) / 2;
-  const long long units = (long long)p.n_pairs * B * Hq;
+  // dense mode with an even group size: a unit is two sibling query heads of one kv head at the
+  // same 128 rows (equal key ranges); otherwise two adjacent row tiles of one head
+  p.sib = (!SPARSE && (Hq / Hkv) % 2 == 0) ? 1 : 0;
+  const long long units = p.sib ? (long long)n_qtiles * B * (Hq / 2) : (long long)p.n_pairs * B * Hq;
   if (units > 0x7fff0000LL) return ATTN_ERR_UNSUPPORTED;  // room for one more round of unit ids
   p.n_units = (int)units;
   // scheduling groups of batches whose K/V (Hkv * Lk rows of d + dv elements each) stays within
@@ -486,11 +490,11 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
   if (d == 128) {
     using C = attn::Prefill2Cfg<128>;
     if (!allow_smem(attn::prefill2_kernel<128, E, SPARSE>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<128, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    attn::prefill2_kernel<128, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, to, p);
   } else {
     using C = attn::Prefill2Cfg<64>;
     if (!allow_smem(attn::prefill2_kernel<64, E, SPARSE>, C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-    attn::prefill2_kernel<64, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, p);
+    attn::prefill2_kernel<64, E, SPARSE><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tq, tk, tv, to, p);
   }
   return launch_status();
 }

@@ -25,7 +25,15 @@
 //     every barrier phase carries across units;
 //   * the block-sparse instantiation (SPARSE) walks the union of the two tiles' caller-given
 //     key-block lists instead of the causal prefix.
-// Warps: 0-7 softmax, 8 TMA producer, 9 TMEM allocator + MMA issuer.
+//   * the output of a tile is written by a separate epilogue warpgroup (warps 8-11): when a
+//     tile's last P is ready, its softmax warpgroup leaves the row statistics in shared memory and
+//     moves on to the next unit, while the epilogue warpgroup waits for the last P.V, reads O out
+//     of TMEM (releasing it for the next unit's first P.V) and stores it through a staging buffer
+//     with TMA. (With the epilogue in the softmax warpgroups the next unit's first P.V waited for
+//     the last P.V, the output stores and a softmax in a row.)
+// Warps: 0-7 softmax, 8-11 epilogue, 12 TMA producer, 13 TMEM allocator + MMA issuer, 14-15 idle.
+// Registers (setmaxnreg): 176 per softmax thread, 64 per epilogue thread, 96 for warps 12-15; at
+// launch 128 each (512 threads), and 2 * 176 + 64 + 96 = 4 * 128.
 #pragma once
 
 #include "sm100.cuh"
@@ -36,8 +44,9 @@ struct Prefill2Params {
   uint16_t* o;  // 16-bit floats of the kernel's element type
   float* lse;
   int B, Hq, Hkv, Lq, Lk, G;
-  int n_pairs;  // ceil(ceil(Lq / 128) / 2)
-  int n_units;  // n_pairs * B * Hq
+  int n_pairs;  // adjacent pairs: ceil(ceil(Lq / 128) / 2)
+  int n_units;  // sibling pairs: n_qblocks * B * Hq / 2; adjacent pairs: n_pairs * B * Hq
+  int sib;      // 1: the two tiles of a unit are query heads h, h + 1 at the same 128 rows
   int group_b;  // batches per scheduling group (their K/V fits comfortably in L2)
   int causal;
   float scale_log2;
@@ -75,13 +84,21 @@ struct Prefill2Cfg {
   static constexpr int NS = (D == 128) ? 2 : 3;
   static constexpr int OFF_Q = 0;  // Q_A, then Q_B
   static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NS * STAGE_BYTES;
-  // q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], o_free[2], drain
-  static constexpr int N_BARS = 2 + 2 * NS + 8 + 1;
+  // Output staging: the epilogue warpgroup writes 64 columns of a tile of O (16-bit, 128-byte
+  // swizzled like Q) here at a time and one of its threads stores them with TMA.
+  static constexpr int OFF_STG = OFF_KV + NS * STAGE_BYTES;
+  // Row statistics (running max m in log2 units, sum l) of each tile's last unit, two buffers
+  // per tile (by the parity of the tile's epilogue count).
+  static constexpr int OFF_STATS = OFF_STG + CHUNK;
+  static constexpr int STATS_BYTES = 2 * 2 * 128 * 8;
+  static constexpr int OFF_BAR = OFF_STATS + STATS_BYTES;
+  // q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], o_free[2], drain,
+  // stats_ready[2 tiles][2 buffers], stg_ready, stg_free
+  static constexpr int N_BARS = 2 + 2 * NS + 8 + 1 + 4 + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 512;
   __host__ __device__ static constexpr uint32_t s_col(int x) { return (uint32_t)(128 * x); }
   __host__ __device__ static constexpr uint32_t o_col(int x) { return (uint32_t)(256 + D * x); }
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -102,6 +119,17 @@ struct UnitCoords {
   int b, h, q0;
 };
 
+// First query row and query head of tile x (0 = A, 1 = B) of a unit. Sibling pairs (dense mode,
+// even group size): heads h and h + 1 of one kv head at the same rows, so both tiles see the same
+// key tiles and finish together. Adjacent pairs: rows q0.. and q0 + 128.. of head h (under a
+// causal mask tile B has one key tile more, which it processes alone).
+__device__ __forceinline__ int tile_row0(const Prefill2Params& p, const UnitCoords& uc, int x) {
+  return uc.q0 + (p.sib ? 0 : 128 * x);
+}
+__device__ __forceinline__ int tile_head(const Prefill2Params& p, const UnitCoords& uc, int x) {
+  return uc.h + (p.sib ? x : 0);
+}
+
 // The key blocks one query tile processes, in increasing order: 0 .. n-1 in dense mode, the
 // caller's list in block-sparse mode.
 struct TileList {
@@ -117,13 +145,13 @@ struct TileList {
 template <bool SPARSE>
 __device__ __forceinline__ TileList prefill_tile_list(const Prefill2Params& p, const UnitCoords& uc, int x,
                                                       bool report) {
-  const int qr0 = uc.q0 + 128 * x;
+  const int qr0 = tile_row0(p, uc, x);
   const int n_dense = prefill_kv_tiles(p, qr0);
   if constexpr (!SPARSE) {
     return TileList{nullptr, n_dense};
   } else {
     if (n_dense == 0) return TileList{nullptr, 0};
-    const long long slot = ((long long)uc.b * p.Hq + uc.h) * p.n_qblocks + qr0 / 128;
+    const long long slot = ((long long)uc.b * p.Hq + tile_head(p, uc, x)) * p.n_qblocks + qr0 / 128;
     const int32_t* lst = p.blk_idx + slot * p.max_blk;
     int cnt = __ldg(p.blk_cnt + slot);
     bool bad = cnt < 0 || cnt > p.max_blk;
@@ -178,24 +206,28 @@ __device__ __forceinline__ int union_size(const TileList& la, const TileList& lb
 }
 
 // Unit order. Batches are taken in groups of group_b whose K/V together fits in L2 with room to
-// spare; within a group the units are sorted by cost (heaviest query-tile pair first: under a
-// causal mask the cost of a pair grows with its position), then by batch, then by head, so that
-// sibling query heads of a kv head are adjacent and share their K/V tiles in L2. (Taking the
+// spare; within a group the units are sorted by cost (heaviest level first: under a causal mask
+// the cost of a unit grows with its rows' position), then by batch, then by head (pair), so that
+// the query heads of a kv head are adjacent and share their K/V tiles in L2. (Taking the
 // heaviest pairs of all batches first would keep every batch's K/V live at once and, for a
 // 16-batch 2K prefill, doubled the DRAM reads.)
 __device__ __forceinline__ UnitCoords prefill_unit(const Prefill2Params& p, int u) {
-  const int per_batch = p.n_pairs * p.Hq;
+  // a level is one 128-row query tile (sibling pairs) or one pair of adjacent tiles, heaviest
+  // first; a level holds one unit per (batch, head pair) or (batch, head)
+  const int n_lvl = p.sib ? p.n_qblocks : p.n_pairs;
+  const int hpl = p.sib ? p.Hq / 2 : p.Hq;
+  const int per_batch = n_lvl * hpl;
   const int per_group = p.group_b * per_batch;
   const int g = u / per_group;
   const int b0 = g * p.group_b;
   const int gb = min(p.group_b, p.B - b0);
   const int w = u - g * per_group;
-  const int lvl = w / (gb * p.Hq);
-  const int rem = w - lvl * gb * p.Hq;
+  const int lvl = w / (gb * hpl);
+  const int rem = w - lvl * gb * hpl;
   UnitCoords c;
-  c.b = b0 + rem / p.Hq;
-  c.h = rem % p.Hq;
-  c.q0 = (p.n_pairs - 1 - lvl) * 256;
+  c.b = b0 + rem / hpl;
+  c.h = (rem % hpl) * (p.sib ? 2 : 1);
+  c.q0 = (n_lvl - 1 - lvl) * (p.sib ? 128 : 256);
   return c;
 }
 
@@ -210,7 +242,8 @@ __device__ __forceinline__ int prefill_unit_index(int k, int cta, int grid) {
 template <int D, typename E, bool SPARSE>
 __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const Prefill2Params p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const Prefill2Params p) {
   using C = Prefill2Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -227,6 +260,12 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
   const uint32_t bar_o_ready = bar_p_full + 16;          // [2]
   const uint32_t bar_o_free = bar_o_ready + 16;          // [2]
   const uint32_t bar_drain = bar_o_free + 16;
+  // one barrier per statistics buffer: a tile whose units have a single key tile can hand over
+  // two units' statistics before the epilogue waits for the first, and a parity wait on a single
+  // barrier could not tell those two phases apart
+  const uint32_t bar_stats_ready = bar_drain + 8;  // [tile * 2 + buffer]
+  const uint32_t bar_stg_ready = bar_stats_ready + 32;
+  const uint32_t bar_stg_free = bar_stg_ready + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
 
   if (threadIdx.x == 0) {
@@ -243,9 +282,12 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       mbar_init(bar_o_free + 8 * x, 128);
     }
     mbar_init(bar_drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar_stats_ready + 8 * i, 128);
+    mbar_init(bar_stg_ready, 128);
+    mbar_init(bar_stg_free, 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
     tc_fence_before();
@@ -253,10 +295,14 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
-
-  if (warp == 8) {
-    // ------------------------------- TMA producer -------------------------------
-    if (lane == 0) {
+  const int wg = warp >> 2;
+  // each role starts with its register reallocation, so that the compiler allocates the role's
+  // code within that role's count
+  if (wg == 3) {
+    regs_decrease<96>();
+    if (warp == 12) {
+      // ------------------------------- TMA producer -------------------------------
+      if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -265,7 +311,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       // stage kv_t % NS receives K and V of one key tile under a single full barrier
       auto load_kv = [&](int tile, int zkv) {
         const int s = kv_t % C::NS;
-        if (kv_t >= C::NS) ok = mbar_wait(bar_kv_empty + 8 * s, ((kv_t / C::NS) & 1) ^ 1, 61);
+        if (kv_t >= C::NS) ok = mbar_wait_inl(bar_kv_empty + 8 * s, ((kv_t / C::NS) & 1) ^ 1, 61);
         if (!ok) return;
         const uint32_t full = bar_kv_full + 8 * s;
         const uint32_t dst = base + C::OFF_KV + s * C::STAGE_BYTES;
@@ -283,18 +329,16 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           const TileList la = prefill_tile_list<SPARSE>(p, uc, 0, true);
           const TileList lb = prefill_tile_list<SPARSE>(p, uc, 1, true);
           if (la.n == 0 && lb.n == 0) continue;  // nothing to load: the softmax writes the empty rows
-          if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
+          if (qc > 0) ok = mbar_wait_inl(bar_q_empty, (qc - 1) & 1, 62);
           if (!ok) break;
-          const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
+          const int zkv = uc.b * p.Hkv + uc.h / p.G;
           mbar_arrive_expect_tx(bar_q_full, ((la.n > 0 ? 1 : 0) + (lb.n > 0 ? 1 : 0)) * C::Q_BYTES);
-          if (la.n > 0) {
-  #pragma unroll
-            for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
-          }
-          if (lb.n > 0) {
+          for (int x = 0; x < 2; ++x) {
+            if ((x == 0 ? la.n : lb.n) == 0) continue;
+            const int zq = uc.b * p.Hq + tile_head(p, uc, x);
   #pragma unroll
             for (int c = 0; c < C::DC; ++c)
-              tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+              tma_load_3d(base + C::OFF_Q + x * C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, tile_row0(p, uc, x), zq);
           }
           ++qc;
           UnionWalk walk(la, lb);
@@ -305,18 +349,17 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       } else {
         for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
           const UnitCoords uc = prefill_unit(p, u);
-          const int nA = prefill_kv_tiles(p, uc.q0), nB = prefill_kv_tiles(p, uc.q0 + 128);
+          const int nA = prefill_kv_tiles(p, tile_row0(p, uc, 0)), nB = prefill_kv_tiles(p, tile_row0(p, uc, 1));
           const int n = max(nA, nB);
-          if (qc > 0) ok = mbar_wait(bar_q_empty, (qc - 1) & 1, 62);
+          if (qc > 0) ok = mbar_wait_inl(bar_q_empty, (qc - 1) & 1, 62);
           if (!ok) break;
-          const int zq = uc.b * p.Hq + uc.h, zkv = uc.b * p.Hkv + uc.h / p.G;
+          const int zkv = uc.b * p.Hkv + uc.h / p.G;
           mbar_arrive_expect_tx(bar_q_full, (nB > 0 ? 2 : 1) * C::Q_BYTES);
-  #pragma unroll
-          for (int c = 0; c < C::DC; ++c) tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0, zq);
-          if (nB > 0) {
+          for (int x = 0; x < (nB > 0 ? 2 : 1); ++x) {
+            const int zq = uc.b * p.Hq + tile_head(p, uc, x);
   #pragma unroll
             for (int c = 0; c < C::DC; ++c)
-              tma_load_3d(base + C::OFF_Q + C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, uc.q0 + 128, zq);
+              tma_load_3d(base + C::OFF_Q + x * C::Q_BYTES + c * C::CHUNK, &tm_q, bar_q_full, 64 * c, tile_row0(p, uc, x), zq);
           }
           ++qc;
           for (int j = 0; j < n && ok; ++j) load_kv(j, zkv);
@@ -327,7 +370,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         for (int u = max(0, kv_t - C::NS); u < kv_t; ++u) mbar_wait_drain(bar_kv_full + 8 * (u % C::NS), (u / C::NS) & 1);
       }
     }
-  } else if (warp == 9) {
+    } else if (warp == 13) {
     // ------------------------------- MMA issuer -------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc(C::BM, C::BN, false, false, E::kFmt);
@@ -336,7 +379,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       int kv_t = 0, qc = 0;
       int p_cnt[2] = {0, 0}, units_done[2] = {0, 0};
       auto wait_stage = [&](int idx, uint32_t site) {
-        ok = mbar_wait(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site);
+        ok = mbar_wait_inl(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site);
         if (ok) tc_fence_after();
       };
       auto issue_s = [&](int x, int sidx) {
@@ -361,7 +404,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           const TileList lx[2] = {prefill_tile_list<SPARSE>(p, uc, 0, false), prefill_tile_list<SPARSE>(p, uc, 1, false)};
           if (lx[0].n == 0 && lx[1].n == 0) continue;
           const int n = union_size<SPARSE>(lx[0], lx[1]);  // key blocks loaded for this unit
-          ok = mbar_wait(bar_q_full, qc & 1, 63);
+          ok = mbar_wait_inl(bar_q_full, qc & 1, 63);
           if (!ok) break;
           ++qc;
           tc_fence_after();
@@ -384,10 +427,10 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             for (int x = 0; x < 2 && ok; ++x) {
               if (in[x]) {
                 if (jx[x] == 0 && units_done[x] > 0) {
-                  ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
+                  ok = mbar_wait_inl(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
                   if (!ok) break;
                 }
-                ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
+                ok = mbar_wait_inl(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
                 if (!ok) break;
                 ++p_cnt[x];
                 tc_fence_after();
@@ -430,10 +473,10 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
           const UnitCoords uc = prefill_unit(p, u);
           int nX[2];
-          nX[0] = prefill_kv_tiles(p, uc.q0);
-          nX[1] = prefill_kv_tiles(p, uc.q0 + 128);
+          nX[0] = prefill_kv_tiles(p, tile_row0(p, uc, 0));
+          nX[1] = prefill_kv_tiles(p, tile_row0(p, uc, 1));
           const int n = max(nX[0], nX[1]);
-          ok = mbar_wait(bar_q_full, qc & 1, 63);
+          ok = mbar_wait_inl(bar_q_full, qc & 1, 63);
           if (!ok) break;
           ++qc;
           tc_fence_after();
@@ -449,10 +492,10 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             for (int x = 0; x < 2 && ok; ++x) {
               if (j >= nX[x]) continue;
               if (j == 0 && units_done[x] > 0) {
-                ok = mbar_wait(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
+                ok = mbar_wait_inl(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
                 if (!ok) break;
               }
-              ok = mbar_wait(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
+              ok = mbar_wait_inl(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
               if (!ok) break;
               ++p_cnt[x];
               tc_fence_after();
@@ -491,7 +534,87 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         mbar_wait_drain(bar_drain, 0);
       }
     }
+    }
+  } else if (wg == 2) {
+    regs_decrease<64>();
+    // ------------------------ epilogue warpgroup (warps 8-11) ------------------------
+    // For each tile with an output, in the order (unit, tile A, tile B): wait for its last P.V and
+    // its row statistics, read O out of TMEM 32 columns at a time (then release O for the next
+    // unit), write O / l as 16-bit rows into the staging buffer and store each 64-column chunk
+    // with TMA; write LSE.
+    const int r = threadIdx.x & 127;  // row of the tile == TMEM lane of this thread
+    const uint32_t tw = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t stg = base + C::OFF_STG;
+    const float2* stats = reinterpret_cast<const float2*>(smem + C::OFF_STATS);
+    int ecnt[2] = {0, 0};  // outputs written per tile
+    int stg_uses = 0;      // chunks stored through the staging buffer
+    bool ok = true;
+    for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
+      const UnitCoords uc = prefill_unit(p, u);
+      for (int x = 0; x < 2 && ok; ++x) {
+        const int qx0 = tile_row0(p, uc, x);
+        if (qx0 >= p.Lq) continue;
+        if (SPARSE && prefill_tile_list<SPARSE>(p, uc, x, false).n == 0) continue;  // written by the softmax
+        const int par = ecnt[x] & 1;
+        ok = mbar_wait_inl(bar_o_ready + 8 * x, par, 70);
+        if (ok) ok = mbar_wait_inl(bar_stats_ready + 8 * (2 * x + par), (ecnt[x] >> 1) & 1, 73);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++ecnt[x];
+        tc_fence_after();
+        const float2 ml = stats[(x * 2 + par) * 128 + r];  // (m in log2 units, l)
+        float inv_l = 1.f / ml.y;
+        if constexpr (SPARSE) inv_l = ml.y > 0.f ? inv_l : 0.f;  // l = 0: the row saw no key
+        const size_t bh = (size_t)uc.b * p.Hq + tile_head(p, uc, x);
+        const uint32_t o_col = C::o_col(x);
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          // columns 32*c4 .. +31: 16-byte units 4*(c4 % 2) .. +3 of the 64-column chunk c4 / 2
+          if ((c4 & 1) == 0 && stg_uses > 0) {
+            ok = mbar_wait_inl(bar_stg_free, (stg_uses - 1) & 1, 71);  // the previous chunk has been read
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+          }
+          float o[32];
+          tmem_ld32(tw + o_col + 32 * c4, o);
+          tmem_wait_ld();
+          if (c4 == D / 32 - 1) {
+            // O has been read out of TMEM: the next unit's first P.V may overwrite it
+            tc_fence_before();
+            mbar_arrive(bar_o_free + 8 * x);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(stg + swz128_offset((uint32_t)r, (uint32_t)(4 * (c4 & 1) + q)),
+                         E::pack2(o[8 * q] * inv_l, o[8 * q + 1] * inv_l), E::pack2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l),
+                         E::pack2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l), E::pack2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
+          if (c4 & 1) {
+            fence_proxy_async_smem();  // the staging writes, visible to the TMA engine
+            mbar_arrive(bar_stg_ready);
+            if (r == 0) {
+              // rows past Lq fall outside the tensor map and are not written
+              if (mbar_wait_inl(bar_stg_ready, stg_uses & 1, 72)) {
+                tma_store_3d(&tm_o, stg, 32 * (c4 - 1), qx0, (int)bh);
+                bulk_commit_group();
+                bulk_wait_read_all();
+              }
+              mbar_arrive(bar_stg_free);
+            }
+            ++stg_uses;
+          }
+        }
+        if (!ok) break;
+        const int row = qx0 + r;
+        if (row < p.Lq && p.lse != nullptr) {
+          float lse_row = (ml.x + log2f(ml.y)) * kLn2;
+          if constexpr (SPARSE) lse_row = ml.y > 0.f ? lse_row : -INFINITY;
+          p.lse[bh * p.Lq + row] = lse_row;
+        }
+      }
+    }
+    if (r == 0) bulk_wait_all();  // this thread's output stores have completed
   } else {
+    regs_increase<176>();
     // --------------------------- softmax warpgroups (warps 0-3: A, 4-7: B) ---------------------------
     const int x = warp >> 2;
     const int r = threadIdx.x & 127;  // row of the tile == TMEM lane
@@ -499,11 +622,12 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     const uint32_t s_col = C::s_col(x), o_col = C::o_col(x);
     const float c2 = p.scale_log2;
     const int off = p.Lk - p.Lq;
-    int s_cnt = 0, o_cnt = 0;
+    int s_cnt = 0, e_cnt = 0;  // S tiles consumed; outputs handed to the epilogue warpgroup
+    float2* stats = reinterpret_cast<float2*>(smem + C::OFF_STATS);
     bool ok = true;
     for (int k = 0, u = blockIdx.x; u < p.n_units && ok; ++k, u = prefill_unit_index(k, blockIdx.x, gridDim.x)) {
       const UnitCoords uc = prefill_unit(p, u);
-      const int qx0 = uc.q0 + 128 * x;
+      const int qx0 = tile_row0(p, uc, x);
       if (qx0 >= p.Lq) continue;  // tile past the last query row
       const TileList lst = prefill_tile_list<SPARSE>(p, uc, x, false);
       const int nt = lst.n;
@@ -511,16 +635,16 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
       if (SPARSE && nt == 0) {
         // no listed block: these rows see no key (O = 0, LSE = -inf); nothing was loaded for them
         if (row < p.Lq) {
-          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + row) * D);
+          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(uc.b * p.Hq + tile_head(p, uc, x)) * p.Lq + row) * D);
 #pragma unroll
           for (int q = 0; q < D / 8; ++q) dst[q] = make_uint4(0u, 0u, 0u, 0u);
-          if (p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = -INFINITY;
+          if (p.lse != nullptr) p.lse[(size_t)(uc.b * p.Hq + tile_head(p, uc, x)) * p.Lq + row] = -INFINITY;
         }
         continue;
       }
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
-        ok = mbar_wait(bar_s_full + 8 * x, s_cnt & 1, 69);
+        ok = mbar_wait_inl(bar_s_full + 8 * x, s_cnt & 1, 69);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++s_cnt;
@@ -611,43 +735,17 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         mbar_arrive(bar_p_full + 8 * x);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16, LSE
-      ok = mbar_wait(bar_o_ready + 8 * x, o_cnt & 1, 70);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ++o_cnt;
-      tc_fence_after();
-      float inv_l = 1.f / l;
-      if constexpr (SPARSE) inv_l = l > 0.f ? inv_l : 0.f;  // l = 0: the row saw no key
-      const bool in_range = row < p.Lq;
-      uint16_t* orow = p.o + ((size_t)(uc.b * p.Hq + uc.h) * p.Lq + (in_range ? row : 0)) * D;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        float o[32];
-        tmem_ld32(tw + o_col + 32 * c4, o);
-        tmem_wait_ld();
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(E::pack2(o[8 * q + 0] * inv_l, o[8 * q + 1] * inv_l),
-                                E::pack2(o[8 * q + 2] * inv_l, o[8 * q + 3] * inv_l),
-                                E::pack2(o[8 * q + 4] * inv_l, o[8 * q + 5] * inv_l),
-                                E::pack2(o[8 * q + 6] * inv_l, o[8 * q + 7] * inv_l));
-        }
-      }
-      if (in_range && p.lse != nullptr) {
-        float lse_row = (m_used + log2f(l)) * kLn2;
-        if constexpr (SPARSE) lse_row = l > 0.f ? lse_row : -INFINITY;
-        p.lse[(size_t)(uc.b * p.Hq + uc.h) * p.Lq + row] = lse_row;
-      }
-      tc_fence_before();
-      mbar_arrive(bar_o_free + 8 * x);
+      // hand the row statistics to the epilogue warpgroup (two buffers: the one written here is
+      // read before the next but one unit of this tile can end, since that unit's first P.V waits
+      // for the epilogue to release O) and go on with the next unit
+      stats[(x * 2 + (e_cnt & 1)) * 128 + r] = make_float2(m_used, l);
+      mbar_arrive(bar_stats_ready + 8 * (2 * x + (e_cnt & 1)));
+      ++e_cnt;
     }
   }
 
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -4,7 +4,10 @@ The kernel's roles are transcribed as generators that yield the barrier waits th
   * the TMA producer (the Q slots of a unit's two query tiles, and a ring of NS stages, stage t
     holding K and V of key tile t under one barrier);
   * the MMA issuer (S = Q.K^T and O += P.V products, commits to the barriers);
-  * the two softmax warpgroups (S -> P in TMEM, the epilogue reading O).
+  * the two softmax warpgroups (S -> P in TMEM; at the end of a unit they leave the row
+    statistics in one of two shared-memory buffers per tile and move on);
+  * the epilogue warpgroup (per output tile: waits for the last P.V and the statistics, reads O
+    out of TMEM and releases it).
 Tensor-core work runs in issue order on a FIFO "pipe"; TMA loads complete in random order. Every
 product checks, when it executes, that the buffers it reads hold the content it expects (the right
 Q tile, K or V tile, P of the right step, O accumulated up to the previous step), so a slot that
@@ -106,12 +109,15 @@ def run(lists, NS, seed, mut=0):
         B[f"p_full{x}"] = Bar(f"p_full{x}")
         B[f"o_ready{x}"] = Bar(f"o_ready{x}")
         B[f"o_free{x}"] = Bar(f"o_free{x}")
+        for b in range(2):
+            B[f"stats_ready{x}{b}"] = Bar(f"stats_ready{x}{b}")
 
     qslot = [None, None]       # ("Q", unit) per slot
     stage = [None] * NS        # ("KV", tile seq) per stage (K and V of one key tile)
     scol = [None, None]        # TMEM S_x columns: ("S" | "P", unit, step)
     ocol = [None, None]        # TMEM O_x: (unit, steps accumulated)
     epi_done = [set(), set()]  # units whose epilogue has read O_x
+    stats = [[None, None], [None, None]]  # per tile, two buffers: the unit whose statistics they hold
     pipe = []                  # FIFO of ("mma", fn) / ("commit", bar)
     tma = []                   # pending loads: (bar, land fn)
     active = [u for u, (la, lb) in enumerate(lists) if la or lb]
@@ -208,7 +214,7 @@ def run(lists, NS, seed, mut=0):
                 next_ready = False
                 for x in range(2):
                     if inn[x]:
-                        if jx[x] == 0 and units_done[x] > 0:
+                        if jx[x] == 0 and units_done[x] > 0 and mut != 8:
                             yield ("wait", f"o_free{x}", (units_done[x] - 1) & 1)
                         yield ("wait", f"p_full{x}", p_cnt[x] & 1)
                         p_cnt[x] += 1
@@ -233,7 +239,7 @@ def run(lists, NS, seed, mut=0):
 
     # ---------------- softmax warpgroups ----------------
     def softmax(x):
-        s_cnt = o_cnt = 0
+        s_cnt = e_cnt = 0
         for u in active:
             nt = len(lists[u][x])
             for j in range(nt):
@@ -247,15 +253,40 @@ def run(lists, NS, seed, mut=0):
                 B[f"p_full{x}"].arrive()
             if nt == 0:
                 continue
-            yield ("wait", f"o_ready{x}", o_cnt & 1)
-            o_cnt += 1
-            if ocol[x] != (u, nt):
-                raise Fail(f"epilogue{x}({u}) reads O holding {ocol[x]}")
-            epi_done[x].add(u)
-            B[f"o_free{x}"].arrive()
+            b = e_cnt & 1 if mut != 6 else 0
+            if stats[x][b] is not None:
+                raise Fail(f"softmax{x}({u}) overwrites the statistics of unit {stats[x][b]} before the epilogue read them")
+            stats[x][b] = u
+            e_cnt += 1
+            B[f"stats_ready{x}{b if mut != 9 else 0}"].arrive()
+
+    # ---------------- epilogue warpgroup ----------------
+    def epilogue():
+        ecnt = [0, 0]
+        for u in active:
+            for x in range(2):
+                nt = len(lists[u][x])
+                if nt == 0:
+                    continue
+                par = ecnt[x] & 1
+                if mut != 7:
+                    yield ("wait", f"o_ready{x}", par)
+                if mut != 9:
+                    yield ("wait", f"stats_ready{x}{par}", (ecnt[x] >> 1) & 1)
+                else:  # one barrier for both buffers: its phases can run two ahead of this wait
+                    yield ("wait", f"stats_ready{x}0", par)
+                ecnt[x] += 1
+                if stats[x][par] != u:
+                    raise Fail(f"epilogue{x}({u}) reads statistics of unit {stats[x][par]}")
+                stats[x][par] = None
+                if ocol[x] != (u, nt):
+                    raise Fail(f"epilogue{x}({u}) reads O holding {ocol[x]}")
+                epi_done[x].add(u)
+                B[f"o_free{x}"].arrive()
 
     consumed = [True, True]
-    roles = {"producer": producer(), "issuer": issuer(), "smA": softmax(0), "smB": softmax(1)}
+    roles = {"producer": producer(), "issuer": issuer(), "smA": softmax(0), "smB": softmax(1),
+             "epilogue": epilogue()}
     waiting = {name: None for name in roles}
     alive = set(roles)
     steps = 0
@@ -289,17 +320,24 @@ def run(lists, NS, seed, mut=0):
     return steps
 
 
-def cta_units(Lq, Hq, batch, grid, cta):
+def cta_units(Lq, Hq, batch, grid, cta, sib=False):
     """One CTA's units in the kernel's order (one scheduling group), as (row0_A, row0_B): pairs of
-    adjacent 128-row tiles, heaviest level first, dealt boustrophedon over `grid` CTAs."""
-    n_pairs = ((Lq + 127) // 128 + 1) // 2
-    n_units = n_pairs * batch * Hq
+    adjacent 128-row tiles of one head, or (sib) the same 128 rows of two sibling heads; heaviest
+    level first, dealt boustrophedon over `grid` CTAs."""
+    n_qt = (Lq + 127) // 128
+    n_lvl = n_qt if sib else (n_qt + 1) // 2
+    hpl = Hq // 2 if sib else Hq
+    n_units = n_lvl * batch * hpl
     out = []
     k, u = 0, cta
     while u < n_units:
-        lvl = u // (batch * Hq)
-        q0 = (n_pairs - 1 - lvl) * 256
-        out.append((q0, q0 + 128))
+        lvl = u // (batch * hpl)
+        if sib:
+            q0 = (n_lvl - 1 - lvl) * 128
+            out.append((q0, q0))
+        else:
+            q0 = (n_lvl - 1 - lvl) * 256
+            out.append((q0, q0 + 128))
         k += 1
         u = k * grid + ((grid - 1 - cta) if (k & 1) else cta)
     return out
@@ -316,24 +354,27 @@ def check(trials=20, geoms=GEOMS, rings=RINGS, mut=0):
     """First failure over dense and sparse runs of the given ring depths and shapes, or None."""
     for NS in rings:
         for geom in geoms:
-            for grid in (1, 3):
-                units = cta_units(geom[0], 2, 2, grid, 0)
+            for grid, sib in ((1, False), (3, False), (1, True), (3, True)):
+                units = cta_units(geom[0], 2, 2, grid, 0, sib)
                 for t in range(trials):
-                    for sparse in (False, True):
+                    for sparse in ((False,) if sib else (False, True)):
                         lists = unit_lists(units, geom, random.Random(1000 + t) if sparse else None)
                         try:
                             run(lists, NS, seed=t, mut=mut)
                         except Fail as e:
-                            return dict(NS=NS, geom=geom, grid=grid, seed=t, sparse=sparse, error=str(e))
+                            return dict(NS=NS, geom=geom, grid=grid, sib=sib, seed=t, sparse=sparse, error=str(e))
     return None
 
 
 # planted slips: 1 a stage never released; 2 a stage released after the first instead of the last
 # P.V of its key tile; 3 the next key tile's S issued without waiting for its stage; 4 a unit's
-# first S issued without waiting for its stage; 5 Q reloaded without waiting for its slot. (Dropping
-# the wait for the previous epilogue is not a slip here: the same threads write the epilogue before
-# they produce the next unit's first P, so P-ready already orders it.)
-MUTANTS = (1, 2, 3, 4, 5)
+# first S issued without waiting for its stage; 5 Q reloaded without waiting for its slot; 6 one
+# statistics buffer per tile instead of two; 7 the epilogue reads O without waiting for the last
+# P.V; 8 the first P.V of a unit issued without waiting for the previous epilogue to release O;
+# 9 one statistics-ready barrier for both buffers of a tile (a tile whose units have a single key
+# tile can then complete two phases before the epilogue waits for the first: a parity wait
+# cannot tell them apart)
+MUTANTS = (1, 2, 3, 4, 5, 6, 7, 8, 9)
 
 
 def mutation_check(trials=20):
