@@ -7,9 +7,10 @@ Llama-3-8B-shaped causal GQA prefill (B=1, Hq=32, Hkv=8, L=8192, d=128): metric 
 (algorithmic flops = 2*(d+dv) per visible query/key pair). The same JSON line also carries the
 MLA-shaped split-KV decode (B=32, 16 heads on one 576/512 latent head, Lq=2, Lk=65536) and the GQA
 decode (B=16, 32 query heads on 8 kv heads, Lk=32768) measured in HBM GB/s, and the fp16-input
-variants of the prefill and of the MLA decode, the 256-token batched prefill (against the larger
-of its compute and HBM times), and the 128K long-context prefill, dense and block-sparse over its
-given index, each with its roofline fraction against MEASURED_PEAKS.json.
+variants of the prefill and of the MLA decode, the 16 x 2K batched causal prefill, the 256-token
+batched prefill (against the larger of its compute and HBM times), and the 128K long-context
+prefill, dense and block-sparse over its given index, each with its roofline fraction against
+MEASURED_PEAKS.json.
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching stream;
 L2 is flushed (a 256 MiB write) before every timed step, outside the events. Multi-GPU (torchrun):
@@ -43,12 +44,28 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # kernels (dram__bytes.sum.per_second x gpu__time_duration.sum; see profiles/): reported as the
 # roofline "traffic". Re-measure whenever one of these kernels changes.
 NCU_TRAFFIC_BYTES = {
-    "llama8b_prefill_8k": 132.6e6,   # prefill2_kernel<128, bf16, dense>
-    "batched_prefill_2k": 787.4e6,   # same kernel
-    "batched_prefill_256": 51.7e6,   # same kernel (O still in L2 when it ends)
+    "llama8b_prefill_8k": 137.6e6,   # prefill2_kernel<128, bf16, dense> (epilogue warpgroup)
+    "batched_prefill_2k": 848.3e6,   # same kernel
+    "batched_prefill_256": 52.6e6,   # same kernel (O still in L2 when it ends)
     "mla_decode_64k": 2427.1e6,      # decode_tn_kernel<9,2,48,3,latent,bf16>, balanced grid
     "gqa_decode_32k": 2154.3e6,      # decode_tn_kernel<2,1,48,3,dense V,bf16>, balanced grid
 }
+# the profiles/ summary each figure above comes from
+NCU_TRAFFIC_SOURCE = {
+    "llama8b_prefill_8k": "profiles/prefill2_kernel_llama8b_prefill_8k.md",
+    "batched_prefill_2k": "profiles/prefill2_kernel_batched_prefill_2k.md",
+    "batched_prefill_256": "profiles/prefill2_kernel_batched_prefill_256.md",
+    "mla_decode_64k": "profiles/decode_tn_kernel_mla_decode_64k.md",
+    "gqa_decode_32k": "profiles/decode_tn_kernel_gqa_decode_32k.md",
+}
+
+
+def traffic(name: str, exact_shape: bool):
+    """(traffic bytes per launch, source) of the profiled kernel for this workload, or (None, None)
+    when this rank's shape is not the profiled one."""
+    if not exact_shape or name not in NCU_TRAFFIC_BYTES:
+        return None, None
+    return NCU_TRAFFIC_BYTES[name], NCU_TRAFFIC_SOURCE[name]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -173,6 +190,16 @@ def job_workload(w, world: int, rank: int, shard: str):
     return w.with_(Hq=sh.Hq, Hkv=sh.Hkv, seed=w.seed + 1000 * rank)
 
 
+def bench_config(w, world: int, shard: str) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+            "dv": w.dv, "causal": w.causal, "flops_per_step_per_gpu": w.flops(),
+            "l2": "flushed (256 MiB write) before every timed step",
+            "parallelism": ("single GPU" if world == 1 else
+                            f"head-sharded x{world} ({w.Hq} query heads per GPU)" if shard == "heads"
+                            else f"independent replicas x{world}")}
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -252,8 +279,39 @@ def bench_prefill_sparse(w, dev, steps, warmup, flush, stream, dense_steps=0):
     return times, pairs, dense_times
 
 
+def host_link_ms(dev, h2d_bytes: int, d2h_bytes: int, reps: int = 5):
+    """Time (ms) to move h2d_bytes host -> device and d2h_bytes device -> host concurrently, as
+    two plain copies on two streams between pinned host memory and the device: the bound of any
+    end-to-end call that moves those bytes over the host link."""
+    hi = torch.empty(h2d_bytes, dtype=torch.uint8, pin_memory=True)
+    ho = torch.empty(d2h_bytes, dtype=torch.uint8, pin_memory=True)
+    di = torch.empty(h2d_bytes, dtype=torch.uint8, device=dev)
+    do = torch.empty(d2h_bytes, dtype=torch.uint8, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    main = torch.cuda.current_stream(dev)
+    best = float("inf")
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        s_in.wait_stream(main)
+        s_out.wait_stream(main)
+        with torch.cuda.stream(s_in):
+            di.copy_(hi, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            ho.copy_(do, non_blocking=True)
+        main.wait_stream(s_in)
+        main.wait_stream(s_out)
+        b.record(main)
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b))
+    return best
+
+
 def bench_prefill_e2e(w, dev, steps, warmup, host):
-    """End to end: pinned host inputs -> device, attn_fwd, O and LSE back to pinned host memory."""
+    """End to end through the library's host entry point (attn_fwd_host): pinned host inputs ->
+    device, the prefill, O and LSE back to pinned host memory, all inside the timed region."""
     from exact_attention_139_b200 import attn
     q, k, v = (t.pin_memory() for t in host)
     bufs = {}
@@ -274,21 +332,25 @@ def bench_prefill_e2e(w, dev, steps, warmup, host):
     return ms, h2d, d2h
 
 
-def bench_decode(w, dev, steps, warmup, flush, stream):
+DECODE_IMPLS = {"auto": 0, "cuda_core": 1, "keys_on_m": 2, "queries_on_m": 3}  # attn_decode_impl
+
+
+def bench_decode(w, dev, steps, warmup, flush, stream, impl="auto", num_splits=0):
+    """Decode steps (split kernel + combine). impl / num_splits select the kernel and the split
+    count (0: the library's own schedule, balanced over the SMs for the tensor-core kernel)."""
     from exact_attention_139_b200 import attn
     q, k, v = make_inputs(w)
     qd, kd = q.to(dev), k.to(dev)
     vd = kd if w.latent else v.to(dev)
     del q, k, v
-    # num_splits = 0: the library's own schedule (balanced over the SMs for the tensor-core kernel);
-    # `splits` reports its partial-slot count
-    splits = attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv)
-    ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, 0),
+    # `splits` reports the partial-slot count
+    splits = num_splits or attn.attn_decode_default_splits(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dv, w.latent)
+    ws = torch.empty(attn.attn_decode_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dv, num_splits),
                      dtype=torch.uint8, device=dev)
     o = torch.empty((w.B, w.Hq, w.Lq, w.dv), dtype=w.torch_dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
-    step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=0,
-                                    workspace=ws, out=o, lse=lse)
+    step = lambda: attn.attn_decode(qd, kd, vd, causal=w.causal, scale=w.scale, dv=w.dv, num_splits=num_splits,
+                                    impl=DECODE_IMPLS[impl], workspace=ws, out=o, lse=lse)
     times = time_steps(step, steps, warmup, flush, stream)
     if attn.attn_check_device() != attn.ATTN_OK:
         raise RuntimeError("device error during the decode benchmark")
@@ -328,15 +390,19 @@ def run_ours(args):
     if not args.no_e2e:
         e_ms, h2d, d2h = bench_prefill_e2e(w, dev, max(2, args.steps // 2), 1, host)
         e_ms = max_over_ranks(e_ms, world)
+        link_ms = host_link_ms(dev, h2d, d2h)
         e2e = {"value": round(flops * world / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)}
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4), "call": "attn_fwd_host (C ABI, host buffers)",
+               "host_link_ms": round(link_ms, 4), "frac_of_host_link": round(link_ms / e_ms, 4)}
     del host
     launches = args.steps  # one prefill kernel per step
     if not args.no_extras:
         wd = job_workload(WORKLOADS["mla_decode_64k"], world, rank, args.shard)
         clocks_d = ClockSampler(torch.cuda.current_device())
         clocks_d.start()
-        dtimes, splits = bench_decode(wd, dev, args.steps, args.warmup, flush, stream)
+        dtimes, splits = bench_decode(wd, dev, args.steps, args.warmup, flush, stream, args.decode_impl,
+                                      args.decode_splits)
+        dflt = args.decode_impl == "auto" and args.decode_splits == 0  # the profiled configuration
         dclk = clocks_d.stop()
         dms = max_over_ranks(sum(dtimes) / len(dtimes), world)
         gbs = wd.kv_bytes() / (dms * 1e-3) / 1e9
@@ -350,16 +416,20 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(ggbs, 1), "peak": float(peaks["hbm_gbs"]),
                          "unit": "GB/s", "frac": round(ggbs / float(peaks["hbm_gbs"]), 4),
                          "algorithmic_bytes_per_launch": wg.kv_bytes(),
-                         "traffic": NCU_TRAFFIC_BYTES.get(wg.name) if wg.Hq == 32 else None}}
+                         "traffic": traffic(wg.name, wg.Hq == 32)[0],
+                         "traffic_source": traffic(wg.name, wg.Hq == 32)[1]}}
         launches += 2 * args.steps
         extras["decode"] = {
             "workload": wd.name, "metric": "KV-read HBM GB/s", "value": round(gbs * world, 1),
-            "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits, "schedule": "balanced grid (num_splits = most partials per kv head)",
-            "kernels_per_step": 2,
+            "per_gpu_gbs": round(gbs, 1), "ms_per_step": round(dms, 4), "num_splits": splits,
+            "schedule": ("balanced grid (num_splits = most partials per kv head)" if args.decode_splits == 0
+                         else f"{args.decode_splits} equal splits per kv head"),
+            "kernel": args.decode_impl, "kernels_per_step": 2,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                          "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": wd.kv_bytes(),
-                         "traffic": NCU_TRAFFIC_BYTES.get(wd.name) if wd.Hq == 16 else None,
+                         "traffic": traffic(wd.name, wd.Hq == 16 and dflt)[0],
+                         "traffic_source": traffic(wd.name, wd.Hq == 16 and dflt)[1],
                          "note": "step = split kernel + combine kernel"},
             "tflops": round(wd.flops() / (dms * 1e-3) / 1e12, 1), "clocks": dclk}
         launches += 2 * args.steps
@@ -376,7 +446,23 @@ def run_ours(args):
             "roofline": {"bound": "max(tensor, hbm)", "achieved_ms": round(shms, 4), "bound_ms": round(t_bound * 1e3, 4),
                          "frac": round(t_bound * 1e3 / shms, 4), "algorithmic_flops_per_launch": wsh.flops(),
                          "algorithmic_bytes_per_launch": sh_bytes,
-                         "traffic": NCU_TRAFFIC_BYTES.get(wsh.name) if world == 1 or args.shard == "batch" else None}}
+                         "traffic": traffic(wsh.name, world == 1 or args.shard == "batch")[0],
+                         "traffic_source": traffic(wsh.name, world == 1 or args.shard == "batch")[1]}}
+        launches += args.steps
+        # batched causal prefill, B = 16 at 2K tokens (the batched configuration of the Llama-3-8B
+        # shape): compute-bound like the 8K prefill, against the same tensor peak
+        wb = job_workload(WORKLOADS["batched_prefill_2k"], world, rank, args.shard)
+        btimes, _ = bench_prefill(wb, dev, args.steps, args.warmup, flush, stream)
+        bms = max_over_ranks(sum(btimes) / len(btimes), world)
+        btf = wb.flops() / (bms * 1e-3) / 1e12
+        b_exact = world == 1 or args.shard == "batch"
+        extras["prefill_batched_2k"] = {
+            "workload": wb.name, "metric": "attention TFLOPS", "value": round(btf * world, 2),
+            "ms_per_step": round(bms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(btf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": round(btf / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "algorithmic_flops_per_launch": wb.flops(),
+                         "traffic": traffic(wb.name, b_exact)[0], "traffic_source": traffic(wb.name, b_exact)[1]}}
         launches += args.steps
         if not args.no_f16:
             # fp16 inputs: same kernels with the fp16 operand format; fp16 and bf16 share one
@@ -432,7 +518,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         rate, nrows, secs, threads = oracle_sample_rate(w, args.cpu_seconds)
         cpu = {"value": round(rate / 1e12, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-               "sample": f"{nrows} seeded query rows of {w.name} (fp64 oracle, {secs:.1f} s)"}
+               "sample": f"{nrows} seeded query rows of {w.name} (fp64 oracle, {secs:.1f} s)",
+               "extrapolated_full_step_s": round(flops / rate, 1)}
 
     if rank == 0:
         line = {
@@ -441,16 +528,12 @@ def run_ours(args):
             "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "strong" if (args.shard == "heads" and world > 1) else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
-                       "dv": w.dv, "causal": w.causal, "flops_per_step_per_gpu": flops,
-                       "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": ("single GPU" if world == 1 else
-                                       f"head-sharded x{world} ({w.Hq} query heads per GPU)" if args.shard == "heads"
-                                       else f"independent replicas x{world}")},
+            "config": bench_config(w, world, args.shard),
             "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": round(per_gpu_tflops / peak_tf, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                          "algorithmic_flops_per_launch": flops,
-                         "traffic": NCU_TRAFFIC_BYTES.get(w.name) if world == 1 or args.shard == "batch" else None},
+                         "traffic": traffic(w.name, world == 1 or args.shard == "batch")[0],
+                         "traffic_source": traffic(w.name, world == 1 or args.shard == "batch")[1]},
             "e2e": e2e,
             "gpu_launches": args.steps,  # one prefill kernel per timed step of the headline leg
             "gpu_launches_all_legs": launches,
@@ -486,10 +569,10 @@ def run_reference(args):
         "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * statistics.mean(step_secs), 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
-                   "dv": w.dv, "causal": w.causal},
+        "config": bench_config(w, 1, "batch"),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_used} seeded query rows per step of {w.name} (fp64 oracle)"},
+                         "sample": f"{rows_used} seeded query rows per step of {w.name} (fp64 oracle)",
+                         "extrapolated_full_step_s": round(w.flops() / (value * 1e12), 1)},
         "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -508,6 +591,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-f16", action="store_true", help="skip the fp16-input measurements")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse prefill measurement")
+    ap.add_argument("--decode-impl", choices=sorted(DECODE_IMPLS), default="auto",
+                    help="kernel of the MLA decode leg (auto: the library's choice, queries on M)")
+    ap.add_argument("--decode-splits", type=int, default=0,
+                    help="split count of the MLA decode leg (0: the library's balanced schedule)")
     ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
                     help="N > 1: each rank runs its own batch (weak scaling) or a head shard of one layer "
                          "(strong scaling, no collective)")
