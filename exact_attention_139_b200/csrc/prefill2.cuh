@@ -372,27 +372,56 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     }
     } else if (warp == 13) {
     // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0) {
+    // The whole warp runs the issuer's control flow and its waits; the lane elected here issues
+    // every product and commit. (Run inside a one-lane branch, the same loop issued M128 products
+    // more slowly than the tensor core retires them; with warp-uniform control flow the issue cost
+    // falls below the math time of a product.)
+    {
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_s = make_idesc(C::BM, C::BN, false, false, E::kFmt);
       constexpr uint32_t idesc_o = make_idesc(C::BM, D, false, true, E::kFmt);
       bool ok = true, issued = false;
       int kv_t = 0, qc = 0;
       int p_cnt[2] = {0, 0}, units_done[2] = {0, 0};
+      // bounded wait by every lane; the outcome is made warp-uniform
+      auto wait_u = [&](uint32_t bar, uint32_t parity, uint32_t site) {
+        ok = __all_sync(0xffffffffu, mbar_wait_inl(bar, parity, site));
+        return ok;
+      };
+      auto commit = [&](uint32_t bar) {
+        if (leader) mma_commit(bar);
+        __syncwarp();
+      };
       auto wait_stage = [&](int idx, uint32_t site) {
-        ok = mbar_wait_inl(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site);
-        if (ok) tc_fence_after();
+        if (wait_u(bar_kv_full + 8 * (idx % C::NS), (idx / C::NS) & 1, site)) tc_fence_after();
       };
       auto issue_s = [&](int x, int sidx) {
         const uint32_t kb = base + C::OFF_KV + (sidx % C::NS) * C::STAGE_BYTES;
         const uint32_t qb = base + C::OFF_Q + x * C::Q_BYTES;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = make_sdesc(qb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          mma_ss(tmem + C::s_col(x), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = make_sdesc(qb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = make_sdesc(kb + (kk >> 2) * C::CHUNK + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+            mma_ss(tmem + C::s_col(x), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_s_full + 8 * x);
         }
-        mma_commit(bar_s_full + 8 * x);
+        __syncwarp();
         issued = true;
+      };
+      // O_x (+)= P_x V of stage si; `first`: the first block of this tile in the unit (overwrite O)
+      auto issue_pv = [&](int x, int si, bool first) {
+        const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
+            // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
+            mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
       };
       // Per key tile j the only wait between the last S product of tile j and the first P.V
       // product of tile j+1 is the one on P: the stage of tile j is released right after its
@@ -404,8 +433,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           const TileList lx[2] = {prefill_tile_list<SPARSE>(p, uc, 0, false), prefill_tile_list<SPARSE>(p, uc, 1, false)};
           if (lx[0].n == 0 && lx[1].n == 0) continue;
           const int n = union_size<SPARSE>(lx[0], lx[1]);  // key blocks loaded for this unit
-          ok = mbar_wait_inl(bar_q_full, qc & 1, 63);
-          if (!ok) break;
+          if (!wait_u(bar_q_full, qc & 1, 63)) break;
           ++qc;
           tc_fence_after();
           UnionWalk walk(lx[0], lx[1]);
@@ -416,8 +444,8 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           if (!ok) break;
           for (int x = 0; x < 2; ++x)
             if (in[x]) issue_s(x, kv_t);
-          if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
-          int jx[2] = {0, 0};                    // blocks of each tile already multiplied by V
+          if (n == 1) commit(bar_q_empty);  // the last S of this unit has been issued
+          int jx[2] = {0, 0};               // blocks of each tile already multiplied by V
           for (int j = 0; j < n && ok; ++j) {
             const int si = kv_t + j;  // stage of union block j
             bool in_next[2] = {false, false};
@@ -426,23 +454,14 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             bool next_ready = false;
             for (int x = 0; x < 2 && ok; ++x) {
               if (in[x]) {
-                if (jx[x] == 0 && units_done[x] > 0) {
-                  ok = mbar_wait_inl(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
-                  if (!ok) break;
-                }
-                ok = mbar_wait_inl(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
-                if (!ok) break;
+                // previous epilogue read O_x
+                if (jx[x] == 0 && units_done[x] > 0 && !wait_u(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66)) break;
+                if (!wait_u(bar_p_full + 8 * x, p_cnt[x] & 1, 67)) break;
                 ++p_cnt[x];
                 tc_fence_after();
-                const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
-  #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                  const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
-                  // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
-                  mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (jx[x] > 0 || kk > 0) ? 1u : 0u);
-                }
+                issue_pv(x, si, jx[x] == 0);
                 // K was last read by the S products of this block (issued earlier), V by this one
-                if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
+                if (x == x_last) commit(bar_kv_empty + 8 * (si % C::NS));
               }
               if (has_next && in_next[x]) {
                 if (!next_ready) {
@@ -454,7 +473,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
               }
               if (in[x]) {
                 if (jx[x] == lx[x].n - 1) {
-                  mma_commit(bar_o_ready + 8 * x);
+                  commit(bar_o_ready + 8 * x);
                   ++units_done[x];
                 }
                 ++jx[x];
@@ -462,7 +481,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
             }
             if (!ok) break;
             // Q may be reloaded once the last S of this unit (issued in step n-2) is done
-            if (j == n - 2) mma_commit(bar_q_empty);
+            if (j == n - 2) commit(bar_q_empty);
             in[0] = in_next[0];
             in[1] = in_next[1];
           }
@@ -476,38 +495,28 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           nX[0] = prefill_kv_tiles(p, tile_row0(p, uc, 0));
           nX[1] = prefill_kv_tiles(p, tile_row0(p, uc, 1));
           const int n = max(nX[0], nX[1]);
-          ok = mbar_wait_inl(bar_q_full, qc & 1, 63);
-          if (!ok) break;
+          if (!wait_u(bar_q_full, qc & 1, 63)) break;
           ++qc;
           tc_fence_after();
           wait_stage(kv_t, 64);  // K_0, V_0
           if (!ok) break;
           for (int x = 0; x < 2; ++x)
             if (nX[x] > 0) issue_s(x, kv_t);
-          if (n == 1) mma_commit(bar_q_empty);  // the last S of this unit has been issued
+          if (n == 1) commit(bar_q_empty);  // the last S of this unit has been issued
           for (int j = 0; j < n && ok; ++j) {
             const int si = kv_t + j;                // stage of tile j
             const int x_last = (j < nX[1]) ? 1 : 0;  // last tile whose P.V reads V_j
             bool next_ready = false;
             for (int x = 0; x < 2 && ok; ++x) {
               if (j >= nX[x]) continue;
-              if (j == 0 && units_done[x] > 0) {
-                ok = mbar_wait_inl(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66);  // previous epilogue read O_x
-                if (!ok) break;
-              }
-              ok = mbar_wait_inl(bar_p_full + 8 * x, p_cnt[x] & 1, 67);
-              if (!ok) break;
+              // previous epilogue read O_x
+              if (j == 0 && units_done[x] > 0 && !wait_u(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66)) break;
+              if (!wait_u(bar_p_full + 8 * x, p_cnt[x] & 1, 67)) break;
               ++p_cnt[x];
               tc_fence_after();
-              const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
-  #pragma unroll
-              for (int kk = 0; kk < C::BN / 16; ++kk) {
-                const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
-                // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
-                mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-              }
+              issue_pv(x, si, j == 0);
               // K_j was last read by S of tile j (issued earlier), V_j by this product
-              if (x == x_last) mma_commit(bar_kv_empty + 8 * (si % C::NS));
+              if (x == x_last) commit(bar_kv_empty + 8 * (si % C::NS));
               if (j + 1 < nX[x]) {
                 if (!next_ready) {
                   wait_stage(si + 1, 68);  // K_{j+1}, V_{j+1}
@@ -517,20 +526,20 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
                 issue_s(x, si + 1);
               }
               if (j == nX[x] - 1) {
-                mma_commit(bar_o_ready + 8 * x);
+                commit(bar_o_ready + 8 * x);
                 ++units_done[x];
               }
             }
             if (!ok) break;
             // Q may be reloaded once the last S of this unit (issued in iteration n-2) is done
-            if (j == n - 2) mma_commit(bar_q_empty);
+            if (j == n - 2) commit(bar_q_empty);
           }
           if (!ok) break;
           kv_t += n;
         }
       }
       if (!ok && issued) {
-        mma_commit(bar_drain);
+        commit(bar_drain);
         mbar_wait_drain(bar_drain, 0);
       }
     }
