@@ -772,7 +772,10 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
     }
   } else if (warp >= 4) {
     // -------------------- S issuers: partial a = chunks a, a + NACC, ... --------------------
-    if (lane == 0) {
+    // Each issuing warp runs its control flow and waits warp-uniformly; its elected lane issues
+    // the products and commits (issuing from inside a one-lane branch is measurably slower).
+    {
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_s = make_idesc(64, BK, false, false, E::kFmt);  // S = Q.K^T
       const int a = warp - 4;
       const uint32_t s_tmem = tmem + (C::S_LANE << 16) + C::S_COL + a * BK;
@@ -782,41 +785,48 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
       for (int g = 0; g < nseg && ok; ++g) {
         const int n_tiles = seg_tiles(g);
         if (n_tiles == 0) continue;
-        ok = mbar_wait(bar_q, qn & 1, 42);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_q, qn & 1, 42));
         if (!ok) break;
         ++qn;
         for (int tt = 0; tt < n_tiles && ok; ++tt, ++t) {
           ok = mbar_wait(bar_kv_full + 8 * (t % NST), (t / NST) & 1, 44);
           // S buffer (t & 1) was last read by the softmax of tile t - 2
           if (ok && t >= 2) ok = mbar_wait(bar_p_full + 8 * (t & 1), ((t - 2) >> 1) & 1, 50);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
           const uint64_t kdesc = make_sdesc(base + C::OFF_KV + (t % NST) * C::STAGE + a * C::KCH, 16, 1024, kSwizzle128B);
           const uint32_t d = s_tmem + (t & 1) * C::NACC * BK;
+          if (leader) {
 #pragma unroll
-          for (int i = 0; i < DCH / C::NACC; ++i) {
+            for (int i = 0; i < DCH / C::NACC; ++i) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              // descriptor start addresses advance by whole 16-byte units
-              const uint64_t qa = qdesc + (uint64_t)((i * C::NACC * C::QCH + ks * 32) >> 4);
-              const uint64_t kb = kdesc + (uint64_t)((i * C::NACC * C::KCH + ks * 32) >> 4);
-              mma_ss(d, qa, kb, idesc_s, (i > 0 || ks > 0) ? 1u : 0u);
+              for (int ks = 0; ks < 4; ++ks) {
+                // descriptor start addresses advance by whole 16-byte units
+                const uint64_t qa = qdesc + (uint64_t)((i * C::NACC * C::QCH + ks * 32) >> 4);
+                const uint64_t kb = kdesc + (uint64_t)((i * C::NACC * C::KCH + ks * 32) >> 4);
+                mma_ss(d, qa, kb, idesc_s, (i > 0 || ks > 0) ? 1u : 0u);
+              }
             }
+            mma_commit(bar_s_full + 8 * (t & 1));
           }
+          __syncwarp();
           issued = true;
-          mma_commit(bar_s_full + 8 * (t & 1));
         }
         if (!ok) break;
-        mma_commit(bar_q_empty);  // this segment's Q may be replaced once these products are done
+        if (leader) mma_commit(bar_q_empty);  // this segment's Q may be replaced once these products are done
+        __syncwarp();
       }
       if (!ok && issued) {
-        mma_commit(bar_drain + 8 * (1 + a));
+        if (leader) mma_commit(bar_drain + 8 * (1 + a));
+        __syncwarp();
         mbar_wait_drain(bar_drain + 8 * (1 + a), 0);
       }
     }
   } else if (warp == 3) {
     // ------------------------------- P.V issuer -------------------------------
-    if (lane == 0) {
+    {
+      const bool leader = elect_one_sync();
       const uint32_t idesc_o = make_idesc(64, NW, false, true, E::kFmt);  // O += P.V
       bool ok = true, issued = false;
       int t = 0, segs_done = 0;
@@ -824,34 +834,38 @@ __global__ void __launch_bounds__(DecodeTnCfg<DCH, NPIECE, BK, NST, SEPV>::THREA
         const int n_tiles = seg_tiles(g);
         if (n_tiles == 0) continue;
         // the first product of a segment overwrites O: the previous segment's O must be read out
-        if (segs_done > 0) ok = mbar_wait(bar_o_free, (segs_done - 1) & 1, 39);
+        if (segs_done > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_free, (segs_done - 1) & 1, 39));
         if (!ok) break;
         for (int tt = 0; tt < n_tiles && ok; ++tt, ++t) {
-          ok = mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43);
+          ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full + 8 * (t & 1), (t >> 1) & 1, 43));
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = base + C::OFF_KV + (t % NST) * C::STAGE + (SEPV ? C::VOFF : 0);  // V rows
           const uint32_t pb = base + C::OFF_P + (t & 1) * C::PB;
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = make_sdesc(pb + kk * 32, 16, 1024, kSwizzle128B);
 #pragma unroll
-            for (int h = 0; h < NPIECE; ++h) {
-              // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
-              const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
-              mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+              for (int h = 0; h < NPIECE; ++h) {
+                // B = V rows of this tile, dv columns [h*NW, h*NW + NW): MN-major, 64-column atoms
+                const uint64_t bd = make_sdesc(kb + (h * NW / 64) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
+                mma_ss(tmem + h * NW, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+              }
             }
+            // the S products of this tile completed before its softmax started, so this commit
+            // also covers every read of the stage
+            mma_commit(bar_kv_empty + 8 * (t % NST));
+            mma_commit(bar_pv_done + 8 * (t & 1));
           }
+          __syncwarp();
           issued = true;
-          // the S products of this tile completed before its softmax started, so this commit
-          // also covers every read of the stage
-          mma_commit(bar_kv_empty + 8 * (t % NST));
-          mma_commit(bar_pv_done + 8 * (t & 1));
         }
         ++segs_done;
       }
       if (!ok && issued) {
-        mma_commit(bar_drain);
+        if (leader) mma_commit(bar_drain);
+        __syncwarp();
         mbar_wait_drain(bar_drain, 0);
       }
     }
