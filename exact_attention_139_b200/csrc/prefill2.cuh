@@ -93,8 +93,8 @@ struct Prefill2Cfg {
   static constexpr int STATS_BYTES = 2 * 2 * 128 * 8;
   static constexpr int OFF_BAR = OFF_STATS + STATS_BYTES;
   // q_full, q_empty, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], o_free[2], drain,
-  // stats_ready[2 tiles][2 buffers], stg_ready, stg_free
-  static constexpr int N_BARS = 2 + 2 * NS + 8 + 1 + 4 + 2;
+  // stats_ready[2 tiles][2 buffers], stg_ready, stg_free, p_half[2]
+  static constexpr int N_BARS = 2 + 2 * NS + 8 + 1 + 4 + 2 + 2;
   static constexpr int OFF_TMEM_SLOT = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_TMEM_SLOT + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -266,6 +266,9 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
   const uint32_t bar_stats_ready = bar_drain + 8;  // [tile * 2 + buffer]
   const uint32_t bar_stg_ready = bar_stats_ready + 32;
   const uint32_t bar_stg_free = bar_stg_ready + 8;
+  // P of a key tile is handed over in two halves (keys 0-63, then 64-127): the first four P.V
+  // products run while the softmax still computes the second half
+  const uint32_t bar_p_half = bar_stg_free + 8;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM_SLOT);
 
   if (threadIdx.x == 0) {
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_s_full + 8 * x, 1);
       mbar_init(bar_p_full + 8 * x, 128);
+      mbar_init(bar_p_half + 8 * x, 128);
       mbar_init(bar_o_ready + 8 * x, 1);
       mbar_init(bar_o_free + 8 * x, 128);
     }
@@ -410,12 +414,13 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         __syncwarp();
         issued = true;
       };
-      // O_x (+)= P_x V of stage si; `first`: the first block of this tile in the unit (overwrite O)
-      auto issue_pv = [&](int x, int si, bool first) {
+      // O_x (+)= P_x V of stage si over keys [64 half, 64 half + 64); `first`: the first block of
+      // this tile in the unit (its first product overwrites O)
+      auto issue_pv = [&](int x, int si, bool first, int half) {
         const uint32_t vb = base + C::OFF_KV + (si % C::NS) * C::STAGE_BYTES + C::KV_BYTES;
         if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
+          for (int kk = half * (C::BN / 32); kk < (half + 1) * (C::BN / 32); ++kk) {
             const uint64_t bd = make_sdesc(vb + kk * 2048, C::CHUNK, 1024, kSwizzle128B);
             // A = P_x in TMEM: keys [16kk, 16kk + 16) are columns [8kk, 8kk + 8) of S_x
             mma_ts(tmem + C::o_col(x), tmem + C::s_col(x) + 8 * kk, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
@@ -456,10 +461,13 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
               if (in[x]) {
                 // previous epilogue read O_x
                 if (jx[x] == 0 && units_done[x] > 0 && !wait_u(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66)) break;
+                if (!wait_u(bar_p_half + 8 * x, p_cnt[x] & 1, 74)) break;
+                tc_fence_after();
+                issue_pv(x, si, jx[x] == 0, 0);
                 if (!wait_u(bar_p_full + 8 * x, p_cnt[x] & 1, 67)) break;
                 ++p_cnt[x];
                 tc_fence_after();
-                issue_pv(x, si, jx[x] == 0);
+                issue_pv(x, si, false, 1);
                 // K was last read by the S products of this block (issued earlier), V by this one
                 if (x == x_last) commit(bar_kv_empty + 8 * (si % C::NS));
               }
@@ -511,10 +519,13 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
               if (j >= nX[x]) continue;
               // previous epilogue read O_x
               if (j == 0 && units_done[x] > 0 && !wait_u(bar_o_free + 8 * x, (units_done[x] - 1) & 1, 66)) break;
+              if (!wait_u(bar_p_half + 8 * x, p_cnt[x] & 1, 74)) break;
+              tc_fence_after();
+              issue_pv(x, si, j == 0, 0);
               if (!wait_u(bar_p_full + 8 * x, p_cnt[x] & 1, 67)) break;
               ++p_cnt[x];
               tc_fence_after();
-              issue_pv(x, si, j == 0);
+              issue_pv(x, si, false, 1);
               // K_j was last read by S of tile j (issued earlier), V_j by this product
               if (x == x_last) commit(bar_kv_empty + 8 * (si % C::NS));
               if (j + 1 < nX[x]) {
@@ -696,6 +707,9 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         }
         const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
         l *= alpha;
+        // a warp that rescales O hands its first half of P over only after the rescale below (the
+        // half barrier waits for all four warps, so no P.V of tile j runs before it)
+        const bool resc = __any_sync(0xffffffffu, rescale);
         // p = 2^(s * c2 - m_ref) on key pairs: packed fma, two ex2, packed sum, bf16x2 pack
         const uint64_t c2x2 = f2_pack(c2, c2), nm2 = f2_pack(-m_ref, -m_ref);
         uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
@@ -721,6 +735,11 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           }
           // P overwrites the S columns it came from: keys 32*q4 .. 32*q4 + 31
           tmem_st16u(tw + s_col + 16 * q4, pk);
+          if (q4 == 1 && !resc) {  // keys 0-63 are in place: the first P.V products may start
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_p_half + 8 * x);
+          }
         }
         float a0, a1, b0, b1;
         f2_unpack(acc0, a0, a1);
@@ -728,7 +747,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         const float sum = (a0 + a1) + (b0 + b1);
         l += sum;
         // s_full of tile j also covers P.V of tile j-1, so O is stable here
-        if (__any_sync(0xffffffffu, rescale)) {
+        if (resc) {
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             float o[32];
@@ -741,6 +760,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
+        if (resc) mbar_arrive(bar_p_half + 8 * x);
         mbar_arrive(bar_p_full + 8 * x);
       }
       if (!ok) break;

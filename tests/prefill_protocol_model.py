@@ -4,8 +4,10 @@ The kernel's roles are transcribed as generators that yield the barrier waits th
   * the TMA producer (the Q slots of a unit's two query tiles, and a ring of NS stages, stage t
     holding K and V of key tile t under one barrier);
   * the MMA issuer (S = Q.K^T and O += P.V products, commits to the barriers);
-  * the two softmax warpgroups (S -> P in TMEM; at the end of a unit they leave the row
-    statistics in one of two shared-memory buffers per tile and move on);
+  * the two softmax warpgroups (S -> P in TMEM, handed over in two halves: keys 0-63 under a
+    half barrier, then all of P; a warpgroup that rescales O hands both over after the rescale; at
+    the end of a unit they leave the row statistics in one of two shared-memory buffers per tile
+    and move on);
   * the epilogue warpgroup (per output tile: waits for the last P.V and the statistics, reads O
     out of TMEM and releases it).
 Tensor-core work runs in issue order on a FIFO "pipe"; TMA loads complete in random order. Every
@@ -107,6 +109,7 @@ def run(lists, NS, seed, mut=0):
     for x in range(2):
         B[f"s_full{x}"] = Bar(f"s_full{x}")
         B[f"p_full{x}"] = Bar(f"p_full{x}")
+        B[f"p_half{x}"] = Bar(f"p_half{x}")
         B[f"o_ready{x}"] = Bar(f"o_ready{x}")
         B[f"o_free{x}"] = Bar(f"o_free{x}")
         for b in range(2):
@@ -114,8 +117,8 @@ def run(lists, NS, seed, mut=0):
 
     qslot = [None, None]       # ("Q", unit) per slot
     stage = [None] * NS        # ("KV", tile seq) per stage (K and V of one key tile)
-    scol = [None, None]        # TMEM S_x columns: ("S" | "P", unit, step)
-    ocol = [None, None]        # TMEM O_x: (unit, steps accumulated)
+    scol = [None, None]        # TMEM S_x columns: ("S" | "Ph" (first half of P) | "P", unit, step)
+    ocol = [None, None]        # TMEM O_x: (unit, steps accumulated, first half of the next step in)
     epi_done = [set(), set()]  # units whose epilogue has read O_x
     stats = [[None, None], [None, None]]  # per tile, two buffers: the unit whose statistics they hold
     pipe = []                  # FIFO of ("mma", fn) / ("commit", bar)
@@ -171,22 +174,27 @@ def run(lists, NS, seed, mut=0):
             pipe.append(("mma", ex))
             pipe.append(("commit", f"s_full{x}"))
 
-        def issue_pv(x, sidx, u, jx):
-            def ex(x=x, sidx=sidx, u=u, jx=jx):
-                if scol[x] is None or scol[x][0] != "P" or scol[x][1] != u:
-                    raise Fail(f"PV{x}({u},{jx}) reads S columns holding {scol[x]}")
+        def issue_pv(x, sidx, u, jx, half):
+            def ex(x=x, sidx=sidx, u=u, jx=jx, half=half):
+                ready = ("Ph", "P") if half == 0 else ("P",)
+                if scol[x] is None or scol[x][0] not in ready or scol[x][1] != u:
+                    raise Fail(f"PV{x}({u},{jx}) half {half} reads S columns holding {scol[x]}")
                 if stage[sidx % NS] != ("KV", sidx):
                     raise Fail(f"PV{x}({u},{jx}) reads stage holding {stage[sidx % NS]}, wants tile {sidx}")
-                if jx == 0:
+                if half == 1:
+                    if ocol[x] != (u, jx, 1):
+                        raise Fail(f"PV{x}({u},{jx}) second half accumulates onto {ocol[x]}")
+                    ocol[x] = (u, jx + 1, 0)
+                    consumed[x] = True
+                elif jx == 0:
                     prev = [w for w in active if w < u and lists[w][x]]
                     if prev and prev[-1] not in epi_done[x]:
                         raise Fail(f"PV{x}({u},0) overwrites O before the epilogue of unit {prev[-1]}")
-                    ocol[x] = (u, 1)
+                    ocol[x] = (u, 0, 1)
                 else:
-                    if ocol[x] != (u, jx):
+                    if ocol[x] != (u, jx, 0):
                         raise Fail(f"PV{x}({u},{jx}) accumulates onto {ocol[x]}")
-                    ocol[x] = (u, jx + 1)
-                consumed[x] = True
+                    ocol[x] = (u, jx, 1)
             pipe.append(("mma", ex))
 
         for u in active:
@@ -216,9 +224,12 @@ def run(lists, NS, seed, mut=0):
                     if inn[x]:
                         if jx[x] == 0 and units_done[x] > 0 and mut != 8:
                             yield ("wait", f"o_free{x}", (units_done[x] - 1) & 1)
-                        yield ("wait", f"p_full{x}", p_cnt[x] & 1)
+                        yield ("wait", f"p_half{x}", p_cnt[x] & 1)
+                        issue_pv(x, si, u, jx[x], 0)
+                        if mut != 10:
+                            yield ("wait", f"p_full{x}", p_cnt[x] & 1)
                         p_cnt[x] += 1
-                        issue_pv(x, si, u, jx[x])
+                        issue_pv(x, si, u, jx[x], 1)
                         if x == x_last and mut != 1:
                             pipe.append(("commit", f"kv_empty{si % NS}"))
                     if in_next[x]:
@@ -247,10 +258,24 @@ def run(lists, NS, seed, mut=0):
                 s_cnt += 1
                 if scol[x] is None or scol[x][:2] != ("S", u):
                     raise Fail(f"softmax{x}({u},{j}) reads {scol[x]}")
-                if j > 0 and rng.random() < 0.3 and ocol[x] != (u, j):
-                    raise Fail(f"softmax{x}({u},{j}) rescales O holding {ocol[x]}")
-                scol[x] = ("P",) + scol[x][1:]
-                B[f"p_full{x}"].arrive()
+                tag = scol[x][1:]
+                if j > 0 and rng.random() < 0.3:
+                    # rescale O after all of P is written, then hand both halves over
+                    scol[x] = ("P",) + tag
+                    if mut == 11:  # the first half handed over before the rescale
+                        B[f"p_half{x}"].arrive()
+                    yield ("step",)
+                    if ocol[x] != (u, j, 0):
+                        raise Fail(f"softmax{x}({u},{j}) rescales O holding {ocol[x]}")
+                    if mut != 11:
+                        B[f"p_half{x}"].arrive()
+                    B[f"p_full{x}"].arrive()
+                else:
+                    scol[x] = ("Ph",) + tag
+                    B[f"p_half{x}"].arrive()
+                    yield ("step",)
+                    scol[x] = ("P",) + tag
+                    B[f"p_full{x}"].arrive()
             if nt == 0:
                 continue
             b = e_cnt & 1 if mut != 6 else 0
@@ -279,7 +304,7 @@ def run(lists, NS, seed, mut=0):
                 if stats[x][par] != u:
                     raise Fail(f"epilogue{x}({u}) reads statistics of unit {stats[x][par]}")
                 stats[x][par] = None
-                if ocol[x] != (u, nt):
+                if ocol[x] != (u, nt, 0):
                     raise Fail(f"epilogue{x}({u}) reads O holding {ocol[x]}")
                 epi_done[x].add(u)
                 B[f"o_free{x}"].arrive()
@@ -293,7 +318,7 @@ def run(lists, NS, seed, mut=0):
     while alive or pipe or tma:
         steps += 1
         choices = [("role", r) for r in sorted(alive)
-                   if waiting[r] is None or B[waiting[r][1]].done(waiting[r][2])]
+                   if waiting[r] is None or waiting[r][0] == "step" or B[waiting[r][1]].done(waiting[r][2])]
         if pipe:
             choices.append(("pipe", None))
         if tma:
@@ -373,8 +398,9 @@ def check(trials=20, geoms=GEOMS, rings=RINGS, mut=0):
 # P.V; 8 the first P.V of a unit issued without waiting for the previous epilogue to release O;
 # 9 one statistics-ready barrier for both buffers of a tile (a tile whose units have a single key
 # tile can then complete two phases before the epilogue waits for the first: a parity wait
-# cannot tell them apart)
-MUTANTS = (1, 2, 3, 4, 5, 6, 7, 8, 9)
+# cannot tell them apart); 10 the second half of a key tile's P.V issued without waiting for all
+# of P; 11 a warpgroup that rescales O hands the first half of P over before the rescale
+MUTANTS = (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11)
 
 
 def mutation_check(trials=20):
