@@ -57,15 +57,18 @@ struct Prefill2Params {
   int max_blk, n_qblocks, n_kblocks;
 };
 
-#ifndef ATTN_EXP2_EMULATE_MASK
-#define ATTN_EXP2_EMULATE_MASK 0x8080u
-#endif
 // Key pairs e (0..15 within each group of 32 keys) whose exponentials are computed with the FMA
-// polynomial (bit e set) instead of ex2.approx on the MUFU unit. One pair in eight measured best
-// on B200 (8K causal prefill: none 1116, 1/8 1135, 1/4 1099, 3/8 1093, 1/2 1071 TFLOP/s; at
-// d = 64, where the exponentials weigh twice as much per tensor product, 1/8 651, 1/4 632,
-// 3/8 609, 1/2 538).
-constexpr uint32_t kExp2EmulateMask = ATTN_EXP2_EMULATE_MASK;
+// polynomial (bit e set) instead of ex2.approx on the MUFU unit. Measured on B200 with the
+// warp-uniform issuer and the split P hand-off (TFLOP/s; 8K causal / 2K batched / 128K / 8K at
+// d = 64): none 1283 / 1053 / 1142 / 722, one pair in sixteen 1293 / 1053 / 1143 / 710, one in
+// eight 1228 / 995 / 1077 / 703, one in four 1137 / 960 / 1003 / 664. (With the earlier one-lane
+// issuer one in eight had been best: the polynomial's extra instructions now cost more than the
+// MUFU time they save.)
+#ifndef ATTN_EXP2_EMULATE_MASK
+#define ATTN_EXP2_EMULATE_MASK(D) ((D) == 64 ? 0x0000u : 0x0080u)
+#endif
+template <int D>
+constexpr uint32_t kExp2EmulateMask = ATTN_EXP2_EMULATE_MASK(D);
 
 // Shared memory: Q_A and Q_B, then a ring of NS stages, stage j holding K_j and V_j under one
 // full and one empty barrier; a stage is released by one commit after the last P.V product of its
@@ -720,7 +723,7 @@ __global__ void __launch_bounds__(Prefill2Cfg<D>::THREADS, 1)
           for (int e = 0; e < 16; ++e) {
             const uint64_t xv = ffma2(f2_pack(s[q4][2 * e], s[q4][2 * e + 1]), c2x2, nm2);
             float p0, p1;
-            if (kExp2EmulateMask & (1u << e)) {
+            if (kExp2EmulateMask<D> & (1u << e)) {
               // this pair on the FMA pipe: the MUFU unit is the softmax's busiest resource
               f2_unpack(exp2_poly2(xv), p0, p1);
             } else {

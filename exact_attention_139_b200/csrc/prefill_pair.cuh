@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
           for (int e = 0; e < 16; ++e) {
             const uint64_t xv = ffma2(f2_pack(s[q4][2 * e], s[q4][2 * e + 1]), c2x2, nm2);
             float p0, p1;
-            if (kExp2EmulateMask & (1u << e)) {
+            if (kExp2EmulateMask<C::D> & (1u << e)) {
               f2_unpack(exp2_poly2(xv), p0, p1);
             } else {
               float x0, x1;
