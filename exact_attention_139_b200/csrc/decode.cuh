@@ -388,49 +388,58 @@ __global__ void __launch_bounds__(DecodeTcCfg<DCH, NB, NP>::THREADS, 1)
     }
   } else if (warp == 5) {
     // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0 && n_tiles > 0) {
+    // warp-uniform control flow and waits; the elected lane issues and commits
+    if (n_tiles > 0) {
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_s = make_idesc(64, NP, false, false, E::kFmt);  // S^T = K.Q^T
       constexpr uint32_t idesc_o = make_idesc(128, NP, true, false, E::kFmt);  // O^T += V^T.P^T
-      bool ok = mbar_wait(bar_q, 0, 22);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, 22));
       bool issued = false;
       auto pv = [&](int tt) {
-        ok = mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 23);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_p_full + 8 * (tt & 1), (tt >> 1) & 1, 23));
         if (!ok) return;
         tc_fence_after();
         const uint32_t kb = base + C::OFF_KV + (tt & 1) * C::STAGE;
         const uint32_t pb = base + C::OFF_P + (tt & 1) * C::PT;
+        if (leader) {
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
+          for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
-          for (int kk = 0; kk < C::BKV / 16; ++kk) {
-            // A = V^T block nb: dv rows [128nb, 128nb+128) = chunks 2nb, 2nb+1 (MN-major)
-            const uint64_t ad = make_sdesc(kb + (2 * nb) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
-            // B = P^T: NP x 64 keys, K-major 8x16B core matrices (LBO 128, SBO 1024)
-            const uint64_t bd = make_sdesc(pb + kk * 256, 128, 1024, kSwizzleNone);
-            mma_ss(tmem + C::O_COL + nb * NP, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < C::BKV / 16; ++kk) {
+              // A = V^T block nb: dv rows [128nb, 128nb+128) = chunks 2nb, 2nb+1 (MN-major)
+              const uint64_t ad = make_sdesc(kb + (2 * nb) * C::KCH + kk * 2048, C::KCH, 1024, kSwizzle128B);
+              // B = P^T: NP x 64 keys, K-major 8x16B core matrices (LBO 128, SBO 1024)
+              const uint64_t bd = make_sdesc(pb + kk * 256, 128, 1024, kSwizzleNone);
+              mma_ss(tmem + C::O_COL + nb * NP, ad, bd, idesc_o, (tt > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          mma_commit(bar_kv_empty + 8 * (tt & 1));
+          mma_commit(bar_pv_done + 8 * (tt & 1));
         }
-        mma_commit(bar_kv_empty + 8 * (tt & 1));
-        mma_commit(bar_pv_done + 8 * (tt & 1));
+        __syncwarp();
       };
       for (int t = 0; t < n_tiles && ok; ++t) {
-        ok = mbar_wait(bar_kv_full + 8 * (t & 1), (t >> 1) & 1, 24);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_kv_full + 8 * (t & 1), (t >> 1) & 1, 24));
         if (!ok) break;
         tc_fence_after();
         const uint32_t kb = base + C::OFF_KV + (t & 1) * C::STAGE;
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 4 * DCH; ++kk) {
-          const uint64_t ad = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-          mma_ss(tmem + C::S_COL + (t & 1) * NP, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4 * DCH; ++kk) {
+            const uint64_t ad = make_sdesc(kb + (kk >> 2) * C::KCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = make_sdesc(base + C::OFF_Q + (kk >> 2) * C::QCH + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+            mma_ss(tmem + C::S_COL + (t & 1) * NP, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_s_full + 8 * (t & 1));
         }
+        __syncwarp();
         issued = true;
-        mma_commit(bar_s_full + 8 * (t & 1));
         if (t > 0) pv(t - 1);
       }
       if (ok) pv(n_tiles - 1);
       if (!ok && issued) {
-        mma_commit(bar_drain);
+        if (leader) mma_commit(bar_drain);
+        __syncwarp();
         mbar_wait_drain(bar_drain, 0);
       }
     }
