@@ -1,4 +1,6 @@
 """attn_fwd (tcgen05 prefill kernel) against the fp64 oracle on the same seeded inputs."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -64,6 +66,68 @@ def test_full_size_every_row(name, per_head, cuda_device):
     o_ref, l_ref = oracle_rows(w, q, k, v, rows)
     og, lg = take_rows(o, lse, rows)
     compare(og, lg, o_ref, l_ref, name)
+
+
+def _ramp_inputs(w: Workload, beta: float):
+    """Inputs that make the lazy O rescale fire in every key tile for half of the warps: query
+    rows alternate by 32 (one warp of a softmax warpgroup) between +u and -u plus N(0, 1) noise,
+    and key t carries beta * t / 128 along u (u = the all-ones direction) plus N(0, 1) noise, so
+    along the keys the + rows' scores climb by beta * sqrt(d) per 128-key tile while the - rows'
+    fall. V is N(0, 1). All draws from one seeded CPU generator, rounded once to bf16."""
+    g = torch.Generator().manual_seed(w.seed)
+    u = torch.ones(w.d)
+    sign = torch.where((torch.arange(w.Lq) // 32) % 2 == 0, 1.0, -1.0)
+    q = torch.randn((w.B, w.Hq, w.Lq, w.d), generator=g) + sign[None, None, :, None] * u
+    ramp = beta * torch.arange(w.Lk, dtype=torch.float32) / 128.0
+    k = torch.randn((w.B, w.Hkv, w.Lk, w.d), generator=g) + ramp[None, None, :, None] * u
+    v = torch.randn((w.B, w.Hkv, w.Lk, w.dv), generator=g)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def _lazy_rescales(w: Workload, q, k, rows):
+    """Per row, how many 128-key tiles after the first raise the row max by more than the lazy
+    threshold (2^8) over the last max used, in fp64 from the bf16 inputs."""
+    qf, kf = q.double(), k.double()
+    G = w.Hq // w.Hkv
+    off = w.Lk - w.Lq
+    out = []
+    for r in rows:
+        b, rem = divmod(int(r), w.Hq * w.Lq)
+        h, i = divmod(rem, w.Lq)
+        s = (kf[b, h // G] @ qf[b, h, i]).numpy() * w.scale * math.log2(math.e)
+        last = min(w.Lk - 1, i + off) if w.causal else w.Lk - 1
+        used, n = None, 0
+        for t0 in range(0, last + 1, 128):
+            m = s[t0:min(last, t0 + 127) + 1].max()
+            if used is None:
+                used = m
+            elif m > used + 8.0:
+                used, n = m, n + 1
+        out.append(n)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 2, 1024, 128, True), (1, 4, 2, 1024, 128, False),
+                                   (1, 3, 1, 1000, 128, True), (1, 4, 2, 1024, 64, True)],
+                         ids=lambda s: "B{}_H{}x{}_L{}_d{}_{}".format(*s[:5], "c" if s[5] else "n"))
+def test_rescale_in_every_tile(shape, cuda_device):
+    """The lazy O rescale in every key tile for the + warps and never for the - warps of each
+    softmax warpgroup, so that within one tile some warps hand the first half of P over early and
+    others only after rescaling O: every row against the oracle (sibling-head units at G = 2,
+    adjacent row tiles at G = 3; causal and not; d = 128 and 64)."""
+    from exact_attention_139_b200 import attn
+    B, Hq, Hkv, L, d, causal = shape
+    w = Workload("rescale", B, Hq, Hkv, L, L, d, d, causal, seed=4242 + L + d)
+    q, k, v = _ramp_inputs(w, beta=1.0 if d == 128 else 1.4)
+    rows = np.arange(B * Hq * L)
+    probe = rows[(rows % L) >= L - 256]  # rows that see at least 6 key tiles
+    n = _lazy_rescales(w, q, k, probe)
+    plus = ((probe % L) // 32) % 2 == 0
+    assert n[plus].min() >= 3 and n[~plus].max() == 0, (n[plus].min(), n[~plus].max())
+    o, lse = attn.attn_fwd(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), causal=causal, scale=w.scale)
+    assert attn.attn_check_device() == 0
+    o_ref, l_ref = oracle_rows(w, q, k, v, rows)
+    compare(o.reshape(-1, d), lse.reshape(-1), o_ref, l_ref, f"rescale {shape}")
 
 
 def test_long_context_sampled(cuda_device):
