@@ -384,6 +384,11 @@ def run_ours(args):
     value = flops * world / (ms * 1e-3) / 1e12
     per_gpu_tflops = flops / (ms * 1e-3) / 1e12
     peak_tf = float(peaks["bf16_tflops"])
+    # kernels that run for milliseconds (the 128K legs: one launch of ~12 ms sparse, ~120 ms dense)
+    # hold the tensor cores busy long enough for the power cap to lower the SM clock, so their
+    # denominator is the sustained figure (a seconds-long GEMM loop) rather than the burst one
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak_tf))
+    sus_src = f"{peak_src} bf16_tflops_sustained (kernel of milliseconds under the power cap)"
 
     extras = {}
     e2e = None
@@ -501,8 +506,9 @@ def run_ours(args):
                 "value": round(stf * world, 2), "ms_per_step": round(sms, 4), "steps": sp_steps,
                 "density": round(pairs / ws_.visible_pairs(), 4),
                 "dense_equivalent_tflops": round(ws_.flops() / (sms * 1e-3) / 1e12, 1),
-                "roofline": {"bound": "tensor", "achieved": round(stf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                             "frac": round(stf / peak_tf, 4), "algorithmic_flops_per_launch": sflops}}
+                "roofline": {"bound": "tensor", "achieved": round(stf, 2), "peak": peak_sus, "unit": "TFLOP/s",
+                             "frac": round(stf / peak_sus, 4), "peak_source": sus_src,
+                             "frac_of_burst": round(stf / peak_tf, 4), "algorithmic_flops_per_launch": sflops}}
             launches += sp_steps
             wl = job_workload(WORKLOADS["long_prefill_128k"], world, rank, args.shard)
             lms = max_over_ranks(sum(ltimes) / len(ltimes), world)
@@ -510,8 +516,9 @@ def run_ours(args):
             extras["prefill_long"] = {
                 "workload": wl.name, "metric": "attention TFLOPS", "value": round(ltf * world, 2),
                 "ms_per_step": round(lms, 3), "steps": long_steps,
-                "roofline": {"bound": "tensor", "achieved": round(ltf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-                             "frac": round(ltf / peak_tf, 4), "algorithmic_flops_per_launch": wl.flops()}}
+                "roofline": {"bound": "tensor", "achieved": round(ltf, 2), "peak": peak_sus, "unit": "TFLOP/s",
+                             "frac": round(ltf / peak_sus, 4), "peak_source": sus_src,
+                             "frac_of_burst": round(ltf / peak_tf, 4), "algorithmic_flops_per_launch": wl.flops()}}
             launches += long_steps
 
     cpu = None
