@@ -44,8 +44,8 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 # kernels (dram__bytes.sum.per_second x gpu__time_duration.sum; see profiles/): reported as the
 # roofline "traffic". Re-measure whenever one of these kernels changes.
 NCU_TRAFFIC_BYTES = {
-    "llama8b_prefill_8k": 137.1e6,   # prefill2_kernel<128, bf16, dense> (warp-uniform issuer, P in halves)
-    "batched_prefill_2k": 813.9e6,   # same kernel
+    "llama8b_prefill_8k": 137.9e6,   # prefill2_kernel<128, bf16, dense> (registers 184 / 64 / 80)
+    "batched_prefill_2k": 839.9e6,   # same kernel
     "batched_prefill_256": 53.8e6,   # same kernel (O still in L2 when it ends)
     "mla_decode_64k": 2421.4e6,      # decode_tn_kernel<9,2,48,3,latent,bf16>, balanced grid
     "gqa_decode_32k": 2150.9e6,      # decode_tn_kernel<2,1,48,3,dense V,bf16>, balanced grid
